@@ -1,0 +1,313 @@
+"""Checks that tie the CPU oracle to facts fixed outside it.
+
+Each check takes the oracle module as an argument so that the mutation tests
+can run the same check against an oracle with a planted mistake and see it
+fail. A check returns None when the pin holds and raises AssertionError
+otherwise. The facts come from the definitions on the pages (pooling means,
+dense softmax attention, online-softmax merge) and from mathematics (brute
+force on tiny inputs, closed forms, invariants); none is a retyped copy of the
+oracle's own formula.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _bf16_exact(x):
+    from workloads import bf16_to_f32, round_bf16
+    return bf16_to_f32(round_bf16(np.asarray(x, dtype=np.float32)))
+
+
+def rand_qkv(seed, B, Hq, Hkv, Nq, N, D):
+    g = _rng(seed)
+    q = _bf16_exact(g.standard_normal((B, Hq, Nq, D)))
+    k = _bf16_exact(g.standard_normal((B, Hkv, N, D)))
+    v = _bf16_exact(g.standard_normal((B, Hkv, N, D)))
+    return q, k, v
+
+
+# ----------------------------------------------------------------------------- P2 pyramid means
+
+def check_pyramid_means(o, seed=7, n_blocks=37, block=16, factor=4, D=24):
+    """Every node equals the fp64 mean of all keys it covers; a node with f full
+    children equals the fp64 mean of its children (ragged tail included)."""
+    g = _rng(seed)
+    keys = _bf16_exact(g.standard_normal((n_blocks * block, D)) * 3.0 + 0.5)
+    levels = o.build_pyramid(keys, block, factor)
+    width = 1
+    for l, lev in enumerate(levels):
+        n_l = -(-n_blocks // width)
+        assert lev.shape == (n_l, D), (l, lev.shape)
+        for c in range(n_l):
+            lo, hi = c * width * block, min((c + 1) * width, n_blocks) * block
+            ref = keys[lo:hi].astype(np.float64).mean(axis=0)
+            assert np.allclose(lev[c], ref, rtol=1e-5, atol=1e-5), (l, c)
+            if l > 0 and (c + 1) * factor <= levels[l - 1].shape[0] and (c + 1) * width <= n_blocks:
+                kids = levels[l - 1][c * factor:(c + 1) * factor].astype(np.float64).mean(axis=0)
+                assert np.allclose(lev[c], kids, rtol=1e-5, atol=1e-5), (l, c)
+        width *= factor
+    assert levels[-1].shape[0] <= factor and (len(levels) == 1 or levels[-2].shape[0] > factor)
+
+
+# ----------------------------------------------------------------------------- query summary
+
+def check_query_summary(o, seed=8):
+    g = _rng(seed)
+    q = _bf16_exact(g.standard_normal((3, 40, 16)))
+    qbar = o.query_summary(q, 8)
+    assert qbar.shape == (5, 16)
+    for i in range(5):
+        ref = q[:, i * 8:(i + 1) * 8].astype(np.float64).reshape(-1, 16).mean(axis=0)
+        assert np.allclose(qbar[i], ref, rtol=1e-6, atol=1e-6), i
+    dec = o.query_summary(q[:, :1], 1)
+    assert np.allclose(dec[0], q[:, 0].astype(np.float64).mean(axis=0), rtol=1e-6, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------- P1 dense reduction
+
+def check_dense_reduction(o, seed=11, causal=True, per_qhead=False, decode=False,
+                          B=1, Hq=4, Hkv=2, N=256, D=32, block=16, factor=4):
+    """With K >= every eligible block, sparse attention is dense softmax attention (fp64 brute force)."""
+    nq = 1 if decode else N
+    q, k, v = rand_qkv(seed, B, Hq, Hkv, nq, N, D)
+    res = o.forward(q, k, v, block, factor, N // block, causal, per_qhead=per_qhead)
+    g = Hq // Hkv
+    scale = 1.0 / math.sqrt(D)
+    for b in range(B):
+        for h in range(Hq):
+            pos = np.full(1, N - 1) if decode else np.arange(N)
+            ref_o, ref_l = o_dense(q[b, h], pos, k[b, h // g], v[b, h // g], causal and not decode, scale)
+            assert np.abs(res["O"][b, h] - ref_o).max() < 1e-5, (b, h)
+            assert np.abs(res["lse"][b, h] - ref_l).max() < 1e-5, (b, h)
+
+
+def o_dense(q, pos, k, v, causal, scale):
+    """Textbook dense attention written out independently of the oracle (fp64)."""
+    s = scale * (q.astype(np.float64) @ k.astype(np.float64).T)
+    if causal:
+        s[np.arange(k.shape[0])[None, :] > pos[:, None]] = -np.inf
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    out = (p @ v.astype(np.float64)) / p.sum(axis=1, keepdims=True)
+    lse = np.log(np.exp(s - s.max(axis=1, keepdims=True)).sum(axis=1)) + s.max(axis=1)
+    return out, lse
+
+
+# ----------------------------------------------------------------------------- P3 cardinality
+
+def check_cardinality(o, seed=12, causal=True, topk=6, N=512, block=16, factor=4):
+    q, k, v = rand_qkv(seed, 1, 2, 1, N, N, 16)
+    res = o.forward(q, k, v, block, factor, topk, causal)
+    nb = N // block
+    for i in range(nb):
+        row = res["idx"][0, 0, i]
+        eligible = i + 1 if causal else nb
+        valid = row[row >= 0]
+        assert len(valid) == min(topk, eligible), (i, row)
+        assert np.all(row[len(valid):] == -1)
+        assert len(set(valid.tolist())) == len(valid)
+        assert np.all(np.diff(valid) > 0)
+        assert valid.max() < eligible and valid.min() >= 0
+
+
+# ----------------------------------------------------------------------------- P4 tie rule
+
+def tie_case():
+    """Key blocks 3, 9 and 12 are identical and point along the query; the rest are zero.
+
+    nb = 16, f = 4, K = 2. At level 1 nodes 0, 2 and 3 tie exactly; the lower
+    indices 0 and 2 are kept, and level 0 then keeps blocks 3 and 9. Exhaustive
+    top-2 with the lower-index rule gives the same {3, 9}.
+    """
+    D, block = 8, 4
+    k = np.zeros((16 * block, D), dtype=np.float32)
+    pattern = np.array([1.0, 0.5, 0, 0, 0, 0, 0, 0], dtype=np.float32)
+    for j in (3, 9, 12):
+        k[j * block:(j + 1) * block] = pattern
+    q = np.zeros((1, block, D), dtype=np.float32)
+    q[0, :, 0] = 1.0
+    return q, k, block, 4, 2, [3, 9]
+
+
+def check_tie_rule(o):
+    q, k, block, factor, topk, expect = tie_case()
+    levels = o.build_pyramid(k, block, factor)
+    qbar = o.query_summary(q, block)[0]
+    r = o.select_blocks(qbar, levels, factor, topk, 15)
+    assert r["idx"] == expect, r["idx"]
+    assert r["margin"] == 0.0
+
+
+# ----------------------------------------------------------------------------- P5/P6 exhaustive
+
+def brute_topk(qbar, k_plane, block, topk, last):
+    """Exhaustive top-K over the eligible level-0 blocks in fp64, lower index on ties; returns (idx, margin)."""
+    nb = k_plane.shape[0] // block
+    means = k_plane.astype(np.float64).reshape(nb, block, -1).mean(axis=1)
+    s = means[:last + 1] @ qbar.astype(np.float64)
+    order = sorted(range(last + 1), key=lambda j: (-s[j], j))
+    if last + 1 <= topk:
+        return sorted(order), math.inf
+    a, b = s[order[topk - 1]], s[order[topk]]
+    return sorted(order[:topk]), (a - b) / max(abs(a), abs(b), 1e-30)
+
+
+def check_full_budgets(o, seed=13, causal=True, N=1024, block=16, factor=4, topk=8, D=16):
+    """Descent with K_l = n_l at every coarse level equals exhaustive top-K at the finest level."""
+    q, k, v = rand_qkv(seed, 1, 2, 1, N, N, D)
+    levels = o.build_pyramid(k[0, 0], block, factor)
+    budgets = [topk] + [lev.shape[0] for lev in levels[1:]]
+    qbar = o.query_summary(q[0], block)
+    nb = N // block
+    checked = 0
+    for i in range(nb):
+        last = i if causal else nb - 1
+        ref, margin = brute_topk(qbar[i], k[0, 0], block, topk, last)
+        if margin < 1e-4:
+            continue
+        got = o.select_blocks(qbar[i], levels, factor, topk, last, budgets)["idx"]
+        assert got == ref, (i, got, ref)
+        checked += 1
+    assert checked > nb // 2
+
+
+def check_single_level(o, seed=14, N=512, block=16, topk=5, D=16):
+    """f >= nb: the pyramid is level 0 alone and the descent is a flat top-K."""
+    q, k, v = rand_qkv(seed, 1, 1, 1, N, N, D)
+    nb = N // block
+    levels = o.build_pyramid(k[0, 0], block, nb)
+    assert len(levels) == 1
+    qbar = o.query_summary(q[0], block)
+    for i in range(nb):
+        ref, margin = brute_topk(qbar[i], k[0, 0], block, topk, nb - 1)
+        if margin < 1e-4:
+            continue
+        assert o.select_blocks(qbar[i], levels, nb, topk, nb - 1)["idx"] == ref
+
+
+# ----------------------------------------------------------------------------- P7 masked dense
+
+def check_masked_dense(o, seed=15, N=256, block=16, D=32, causal=True):
+    """Attention over chosen blocks equals fp64 dense attention with -inf outside those blocks."""
+    q, k, v = rand_qkv(seed, 1, 1, 1, N, N, D)
+    g = _rng(seed + 1)
+    scale = 1.0 / math.sqrt(D)
+    for i in (0, 3, 15):
+        blocks = sorted(set(g.choice(i + 1, size=min(4, i + 1), replace=False).tolist()) | {i})
+        rows = np.arange(i * block, (i + 1) * block)
+        out, lse = o.attend(q[0, 0, rows], rows, k[0, 0], v[0, 0], blocks, block, causal, scale)
+        allowed = np.zeros((block, N), dtype=bool)
+        for j in blocks:
+            allowed[:, j * block:(j + 1) * block] = True
+        s = scale * (q[0, 0, rows].astype(np.float64) @ k[0, 0].astype(np.float64).T)
+        keep = allowed & (np.arange(N)[None, :] <= rows[:, None] if causal else True)
+        s = np.where(keep, s, -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        ref = (p @ v[0, 0].astype(np.float64)) / p.sum(axis=1, keepdims=True)
+        assert np.abs(out - ref).max() < 1e-5, i
+        ref_lse = s.max(axis=1) + np.log(p.sum(axis=1))
+        assert np.abs(lse - ref_lse).max() < 1e-5, i
+
+
+# ----------------------------------------------------------------------------- P8 merge
+
+def check_merge(o, seed=16, N=512, block=16, D=32):
+    """Splitting the selected blocks into parts and merging by LSE equals the unsplit result."""
+    q, k, v = rand_qkv(seed, 1, 1, 1, N, N, D)
+    rows = np.arange(20 * block, 21 * block)
+    blocks = [1, 4, 7, 8, 13, 19, 20]
+    scale = 1.0 / math.sqrt(D)
+    full_o, full_l = o.attend(q[0, 0, rows], rows, k[0, 0], v[0, 0], blocks, block, True, scale)
+    for parts in ([[1, 4], [7, 8, 13], [19, 20]], [[1], [4, 7, 8, 13, 19, 20]], [[20], [1, 4, 7], [8], [13, 19]]):
+        outs, lses = zip(*[o.attend(q[0, 0, rows], rows, k[0, 0], v[0, 0], p, block, True, scale) for p in parts])
+        mo, ml = o.merge_partials(list(outs), list(lses))
+        assert np.abs(mo - full_o).max() < 1e-5
+        assert np.abs(ml - full_l).max() < 1e-5
+    # a partial whose rows are all masked carries lse = -inf and weight 0
+    lse_a = np.array([0.3, -1.0]); lse_b = np.array([1.2, 0.5])
+    oa = np.array([[1.0, 0.0], [0.0, 2.0]]); ob = np.array([[0.0, 1.0], [4.0, 0.0]])
+    mo, ml = o.merge_partials([oa, ob], [lse_a, lse_b])
+    wa = np.exp(lse_a) / (np.exp(lse_a) + np.exp(lse_b))
+    assert np.allclose(mo, wa[:, None] * oa + (1 - wa)[:, None] * ob, atol=1e-12)
+    assert np.allclose(ml, np.log(np.exp(lse_a) + np.exp(lse_b)), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- causality (R6)
+
+def check_causal_partial_node(o, seed=17, N=1024, block=16, factor=4, D=16):
+    """A node straddling the query block is summarised by the mean of its eligible keys only."""
+    g = _rng(seed)
+    k = _bf16_exact(g.standard_normal((N, D)))
+    levels = o.build_pyramid(k, block, factor)
+    nb = N // block
+    for last in (0, 5, 17, 33, 62):
+        for l in range(len(levels)):
+            width = factor ** l
+            c = last // width
+            lo = c * width
+            hi = min((c + 1) * width, nb) - 1
+            ref = k[lo * block:(last + 1) * block].astype(np.float64).mean(axis=0)
+            got = o.node_value(levels, factor, l, c, last)
+            assert np.allclose(got, ref, rtol=1e-5, atol=1e-5), (last, l)
+            if hi <= last:
+                assert np.array_equal(got, levels[l][c])
+
+
+def check_causal_invariance(o, seed=18, N=1024, block=16, factor=4, topk=5, D=16):
+    """Changing keys after a query block changes neither its selection nor its output."""
+    q, k, v = rand_qkv(seed, 1, 2, 1, N, N, D)
+    base = o.forward(q, k, v, block, factor, topk, True)
+    i = 21
+    k2, v2 = k.copy(), v.copy()
+    g = _rng(seed + 5)
+    k2[0, 0, (i + 1) * block:] = _bf16_exact(g.standard_normal(((N // block - i - 1) * block, D)) * 4)
+    v2[0, 0, (i + 1) * block:] = _bf16_exact(g.standard_normal(((N // block - i - 1) * block, D)))
+    # plant a strong future block: a leak through a straddling node would pull its parent in
+    k2[0, 0, (i + 2) * block:(i + 3) * block] = 50.0 * q[0].mean(axis=(0, 1))[None, :]
+    alt = o.forward(q, k2, v2, block, factor, topk, True)
+    for j in range(i + 1):
+        assert np.array_equal(base["idx"][0, 0, j], alt["idx"][0, 0, j]), j
+    rows = slice(0, (i + 1) * block)
+    assert np.array_equal(base["O"][0, :, rows], alt["O"][0, :, rows])
+
+
+# ----------------------------------------------------------------------------- P10 work bound
+
+def check_work_bound(o, seed=19, N=4096, block=16, factor=4, topk=8, D=16):
+    """Candidates scored per query block stay within n_top + sum_l K_l f (O(N log N))."""
+    q, k, v = rand_qkv(seed, 1, 1, 1, N, N, D)
+    levels = o.build_pyramid(k[0, 0], block, factor)
+    qbar = o.query_summary(q[0], block)
+    bound = levels[-1].shape[0] + (len(levels) - 1) * topk * factor
+    nb = N // block
+    for i in (0, 7, 100, nb - 1):
+        r = o.select_blocks(qbar[i], levels, factor, topk, i)
+        assert r["n_scored"] <= bound, (i, r["n_scored"], bound)
+    r = o.select_blocks(qbar[nb - 1], levels, factor, topk, nb - 1)
+    assert r["n_scored"] < nb
+
+
+ALL_PINS = {
+    "pyramid_means": check_pyramid_means,
+    "query_summary": check_query_summary,
+    "dense_reduction_causal": lambda o: check_dense_reduction(o, causal=True),
+    "dense_reduction_noncausal": lambda o: check_dense_reduction(o, causal=False, Hq=2, Hkv=2),
+    "dense_reduction_per_qhead": lambda o: check_dense_reduction(o, causal=True, per_qhead=True),
+    "dense_reduction_decode": lambda o: check_dense_reduction(o, decode=True, B=2),
+    "cardinality_causal": lambda o: check_cardinality(o, causal=True),
+    "cardinality_noncausal": lambda o: check_cardinality(o, causal=False),
+    "tie_rule": check_tie_rule,
+    "full_budgets_causal": lambda o: check_full_budgets(o, causal=True),
+    "full_budgets_noncausal": lambda o: check_full_budgets(o, causal=False),
+    "single_level": check_single_level,
+    "masked_dense": check_masked_dense,
+    "merge": check_merge,
+    "causal_partial_node": check_causal_partial_node,
+    "causal_invariance": check_causal_invariance,
+    "work_bound": check_work_bound,
+}

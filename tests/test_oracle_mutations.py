@@ -1,0 +1,105 @@
+"""Planted mistakes in the oracle must each fail at least one pin.
+
+Each mutation patches one oracle function on the CPU with a plausible slip (a
+dropped term, a wrong sign, an off-by-one index, a swapped operand) and runs
+the pins; the test passes when some pin raises. This shows the pins can see
+mistakes in every step, not only that the current oracle passes them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import pisa_oracle as po
+from tests import pins
+
+F32 = np.float32
+_orig_children = po.children
+_orig_block_means = po.block_means
+_orig_attend = po.attend
+_orig_node_value = po.node_value
+_orig_query_summary = po.query_summary
+_orig_merge = po.merge_partials
+_orig_level_sizes = po.level_sizes
+
+
+def _drop_last_child(n_below, factor, c):
+    return list(range(c * factor, min(c * factor + factor - 1, n_below)))
+
+
+def _mean_off_by_one(k_plane, block):
+    n0 = k_plane.shape[0] // block
+    return k_plane[:n0 * block].astype(F32).reshape(n0, block, -1).sum(axis=1) / F32(block + 1)
+
+
+def _rank_ascending(score_value, node):
+    return (float(score_value), node)
+
+
+def _rank_ties_high(score_value, node):
+    return (-float(score_value), -node)
+
+
+def _attend_causal_strict(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale):
+    return _orig_attend(q_rows, q_pos - 1, k_plane, v_plane, blocks, block, causal, scale)
+
+
+def _attend_no_scale(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale):
+    return _orig_attend(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, 1.0)
+
+
+def _attend_values_swapped(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale):
+    return _orig_attend(q_rows, q_pos, v_plane, k_plane, blocks, block, causal, scale)
+
+
+def _node_value_leaky(levels, factor, level, c, last):
+    return levels[level][c]
+
+
+def _query_first_head(q_heads, rows_per_block):
+    return _orig_query_summary(q_heads[:1], rows_per_block)
+
+
+def _merge_wrong_sign(outs, lses):
+    return _orig_merge(outs, [-x for x in lses])
+
+
+def _score_dropped_component(qbar, node):
+    return F32(np.dot(qbar[1:].astype(F32), node[1:].astype(F32)))
+
+
+def _one_level_too_many(n0, factor):
+    sizes = [n0]
+    while sizes[-1] >= factor:
+        sizes.append(-(-sizes[-1] // factor))
+    return sizes
+
+
+MUTATIONS = {
+    "pyramid drops a child": ("children", _drop_last_child),
+    "level-0 mean divides by block+1": ("block_means", _mean_off_by_one),
+    "selection keeps the lowest scores": ("rank_key", _rank_ascending),
+    "ties go to the higher index": ("rank_key", _rank_ties_high),
+    "causal mask excludes the diagonal key": ("attend", _attend_causal_strict),
+    "softmax scale dropped": ("attend", _attend_no_scale),
+    "K and V swapped": ("attend", _attend_values_swapped),
+    "straddling node leaks future keys": ("node_value", _node_value_leaky),
+    "query summary uses one head of the group": ("query_summary", _query_first_head),
+    "merge weights with the wrong sign": ("merge_partials", _merge_wrong_sign),
+    "score drops one component": ("score", _score_dropped_component),
+    "pyramid builds one level too many": ("level_sizes", _one_level_too_many),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, bad = MUTATIONS[name]
+    monkeypatch.setattr(po, attr, bad)
+    failed = []
+    for pin_name, pin in pins.ALL_PINS.items():
+        try:
+            pin(po)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin_name)
+    assert failed, f"no pin caught: {name}"
