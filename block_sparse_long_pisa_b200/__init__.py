@@ -1,0 +1,319 @@
+"""Python binding of libpisa.so (PISA pyramid block-sparse attention for B200).
+
+Argument marshalling only: every step of the method runs in the CUDA kernels
+behind the C ABI of include/pisa.h. PyTorch supplies device memory and the
+current stream. There is no CPU fallback: importing this package fails if the
+compiled library is missing, and every call raises PisaError on a non-OK
+status.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpisa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libpisa.so is not built ({LIB_PATH}); run __graft_entry__.build() first")
+_lib = ctypes.CDLL(LIB_PATH)
+
+MAX_LEVELS = 24
+MAX_CANDIDATES = 4096
+
+STATUS = {0: "PISA_OK", 1: "PISA_ERR_INVALID_ARG", 2: "PISA_ERR_UNSUPPORTED", 3: "PISA_ERR_WORKSPACE",
+          4: "PISA_ERR_CUDA", 5: "PISA_ERR_TIMEOUT", 6: "PISA_ERR_BAD_INDEX"}
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_BAD_INDEX = range(7)
+
+
+class PisaShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads_q", "heads_kv", "seq_q", "seq_kv", "head_dim",
+                                               "block", "factor", "topk", "causal", "select_per_qhead")] + \
+               [("scale", ctypes.c_float)]
+
+
+class PisaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: int | None = None):
+        self.status = status
+        self.detail = detail
+        msg = f"{where}: {STATUS.get(status, status)} ({_lib.pisa_status_string(status).decode()})"
+        if detail is not None:
+            msg += f" detail=0x{detail:x}"
+        super().__init__(msg)
+
+
+_vp, _i32p, _f32p, _szp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)
+_SP = ctypes.POINTER(PisaShape)
+_sig = {
+    "pisa_num_levels": (ctypes.c_int32, [_SP]),
+    "pisa_level_layout": (ctypes.c_int, [_SP, _i32p, _i32p]),
+    "pisa_pyramid_size": (ctypes.c_int, [_SP, _szp]),
+    "pisa_workspace_size": (ctypes.c_int, [_SP, _szp]),
+    "pisa_build_pyramid": (ctypes.c_int, [_SP, _vp, _vp, _vp]),
+    "pisa_select_blocks": (ctypes.c_int, [_SP, _vp, _vp, _i32p, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "pisa_sparse_attention": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "pisa_forward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "pisa_check_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
+    "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "pisa_last_launch_count": (ctypes.c_int32, []),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_sig)
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    """Problem description (mirrors pisa_shape)."""
+    batch: int
+    heads_q: int
+    heads_kv: int
+    seq_q: int
+    seq_kv: int
+    head_dim: int
+    block: int
+    factor: int
+    topk: int
+    causal: int = 0
+    select_per_qhead: int = 0
+    scale: float = 0.0
+
+    def c(self) -> PisaShape:
+        return PisaShape(self.batch, self.heads_q, self.heads_kv, self.seq_q, self.seq_kv, self.head_dim,
+                         self.block, self.factor, self.topk, int(self.causal), int(self.select_per_qhead),
+                         float(self.scale))
+
+    @property
+    def decode(self) -> bool:
+        return self.seq_q == 1
+
+    @property
+    def n_blocks(self) -> int:
+        return self.seq_kv // self.block
+
+    @property
+    def hsel(self) -> int:
+        return self.heads_q if self.select_per_qhead else self.heads_kv
+
+    @property
+    def n_qblocks(self) -> int:
+        return 1 if self.decode else self.seq_q // self.block
+
+    @classmethod
+    def of(cls, w, **kw) -> "Shape":
+        """Shape of a workload description (any object with the same field names)."""
+        f = {k: getattr(w, k) for k in ("batch", "heads_q", "heads_kv", "seq_q", "seq_kv", "head_dim", "block",
+                                        "factor", "topk", "causal")}
+        f.update(kw)
+        return cls(**f)
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise PisaError(status, where)
+
+
+def num_levels(shape: Shape) -> int:
+    return int(_lib.pisa_num_levels(ctypes.byref(shape.c())))
+
+
+def level_layout(shape: Shape) -> tuple[list[int], list[int]]:
+    sizes = (ctypes.c_int32 * MAX_LEVELS)()
+    offs = (ctypes.c_int32 * MAX_LEVELS)()
+    _check(_lib.pisa_level_layout(ctypes.byref(shape.c()), sizes, offs), "pisa_level_layout")
+    n = num_levels(shape)
+    return list(sizes[:n]), list(offs[:n])
+
+
+def pyramid_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.pisa_pyramid_size(ctypes.byref(shape.c()), ctypes.byref(n)), "pisa_pyramid_size")
+    return n.value
+
+
+def workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.pisa_workspace_size(ctypes.byref(shape.c()), ctypes.byref(n)), "pisa_workspace_size")
+    return n.value
+
+
+def last_launch_count() -> int:
+    return int(_lib.pisa_last_launch_count())
+
+
+# ----------------------------------------------------------------------------- torch-facing calls
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t, dtype, shape, name):
+    torch = _torch()
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def new_workspace(shape: Shape, device) -> "object":
+    """Zeroed workspace (the status word must start at zero)."""
+    torch = _torch()
+    return torch.zeros(workspace_size(shape), dtype=torch.uint8, device=device)
+
+
+def build_pyramid(shape: Shape, K, pyramid=None, stream=None):
+    torch = _torch()
+    D = shape.head_dim
+    _need(K, torch.bfloat16, (shape.batch, shape.heads_kv, shape.seq_kv, D), "K")
+    sizes, _ = level_layout(shape)
+    if pyramid is None:
+        pyramid = torch.empty((shape.batch, shape.heads_kv, sum(sizes), D), dtype=torch.float32, device=K.device)
+    _check(_lib.pisa_build_pyramid(ctypes.byref(shape.c()), _ptr(K), _ptr(pyramid), _stream(stream)),
+           "pisa_build_pyramid")
+    return pyramid
+
+
+def select_blocks(shape: Shape, Q, pyramid, ws, level_budget=None, idx=None, margin=False, stream=None):
+    torch = _torch()
+    _need(Q, torch.bfloat16, (shape.batch, shape.heads_q, shape.seq_q, shape.head_dim), "Q")
+    if idx is None:
+        idx = torch.empty((shape.batch, shape.hsel, shape.n_qblocks, shape.topk), dtype=torch.int32, device=Q.device)
+    marg = torch.empty((shape.batch, shape.hsel, shape.n_qblocks), dtype=torch.float32, device=Q.device) \
+        if margin else None
+    budget = None
+    if level_budget is not None:
+        budget = (ctypes.c_int32 * len(level_budget))(*[int(x) for x in level_budget])
+    _check(_lib.pisa_select_blocks(ctypes.byref(shape.c()), _ptr(Q), _ptr(pyramid), budget, _ptr(idx), _ptr(marg),
+                                   _ptr(ws), ws.numel(), _stream(stream)), "pisa_select_blocks")
+    return (idx, marg) if margin else idx
+
+
+def sparse_attention(shape: Shape, Q, K, V, idx, ws, O=None, lse=True, stream=None):
+    torch = _torch()
+    B, Hq, Nq, D = shape.batch, shape.heads_q, shape.seq_q, shape.head_dim
+    _need(Q, torch.bfloat16, (B, Hq, Nq, D), "Q")
+    if O is None:
+        O = torch.empty_like(Q)
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else (lse or None)
+    _check(_lib.pisa_sparse_attention(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O),
+                                      _ptr(L), _ptr(ws), ws.numel(), _stream(stream)), "pisa_sparse_attention")
+    return O, L
+
+
+def forward(shape: Shape, Q, K, V, ws, O=None, lse=True, idx=None, stream=None):
+    """Pyramid, selection and attention in one call. Returns (O, lse, idx or None)."""
+    torch = _torch()
+    B, Hq, Nq, D = shape.batch, shape.heads_q, shape.seq_q, shape.head_dim
+    _need(Q, torch.bfloat16, (B, Hq, Nq, D), "Q")
+    _need(K, torch.bfloat16, (B, shape.heads_kv, shape.seq_kv, D), "K")
+    _need(V, torch.bfloat16, (B, shape.heads_kv, shape.seq_kv, D), "V")
+    if O is None:
+        O = torch.empty_like(Q)
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else (lse or None)
+    if idx is True:
+        idx = torch.empty((B, shape.hsel, shape.n_qblocks, shape.topk), dtype=torch.int32, device=Q.device)
+    _check(_lib.pisa_forward(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(L), _ptr(idx),
+                             _ptr(ws), ws.numel(), _stream(stream)), "pisa_forward")
+    return O, L, idx
+
+
+def check_status(ws, stream=None) -> tuple[int, int]:
+    """Synchronises the stream; returns (status, detail) recorded by kernels and clears them."""
+    detail = ctypes.c_uint32()
+    st = _lib.pisa_check_status(_ptr(ws), ctypes.byref(detail), _stream(stream))
+    return int(st), int(detail.value)
+
+
+def raise_on_device_error(ws, where="device", stream=None) -> None:
+    st, detail = check_status(ws, stream)
+    if st != OK:
+        raise PisaError(st, where, detail)
+
+
+class Session:
+    """Preallocated device buffers for repeated forwards of one shape.
+
+    `forward` accepts host (CPU, ideally pinned) or device tensors. Host inputs
+    are copied to the device on the current stream, the pyramid, selection and
+    attention run in the library, and O is copied back into a host tensor.
+    """
+
+    def __init__(self, shape: Shape, device="cuda"):
+        torch = _torch()
+        self.shape = shape
+        self.device = torch.device(device)
+        s = shape
+        self.ws = new_workspace(shape, self.device)
+        self.q = torch.empty((s.batch, s.heads_q, s.seq_q, s.head_dim), dtype=torch.bfloat16, device=self.device)
+        self.k = torch.empty((s.batch, s.heads_kv, s.seq_kv, s.head_dim), dtype=torch.bfloat16, device=self.device)
+        self.v = torch.empty_like(self.k)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((s.batch, s.heads_q, s.seq_q), dtype=torch.float32, device=self.device)
+
+    def forward(self, Q, K, V, out=None):
+        on_host = not Q.is_cuda
+        if on_host:
+            self.q.copy_(Q, non_blocking=True)
+            self.k.copy_(K, non_blocking=True)
+            self.v.copy_(V, non_blocking=True)
+            Q, K, V = self.q, self.k, self.v
+        O, L, _ = forward(self.shape, Q, K, V, self.ws, O=self.o, lse=self.lse)
+        if on_host:
+            if out is None:
+                out = _torch().empty(tuple(O.shape), dtype=O.dtype, pin_memory=True)
+            out.copy_(O, non_blocking=True)
+            return out
+        return O
+
+
+# ----------------------------------------------------------------------------- measurement helpers
+
+def attention_pairs(idx: np.ndarray, shape: Shape) -> int:
+    """Unmasked (query, key) pairs the attention evaluates for a selection (host arithmetic).
+
+    A selected block j < i contributes b*b pairs per query head, the diagonal
+    block (causal) b(b+1)/2; decode contributes b per selected block per head.
+    """
+    b = shape.block
+    heads_per_row = 1 if shape.select_per_qhead else shape.heads_q // shape.heads_kv
+    valid = idx >= 0
+    if shape.decode:
+        return int(valid.sum()) * b * heads_per_row
+    full = int(valid.sum()) * b * b
+    if shape.causal:
+        i = np.arange(idx.shape[2]).reshape(1, 1, -1, 1)
+        diag = int(((idx == i) & valid).sum())
+        full -= diag * (b * b - b * (b + 1) // 2)
+    return full * heads_per_row
+
+
+def attention_flops(idx: np.ndarray, shape: Shape) -> float:
+    """Algorithmic FLOPs of the attention step: 4 * D per unmasked (query, key) pair (QK^T and PV)."""
+    return 4.0 * shape.head_dim * attention_pairs(idx, shape)
+
+
+def default_scale(shape: Shape) -> float:
+    return shape.scale if shape.scale > 0 else 1.0 / math.sqrt(shape.head_dim)

@@ -1,0 +1,388 @@
+// Host side of the C ABI declared in include/pisa.h: argument checks (which
+// never touch the GPU), workspace layout and the launch sequence of every call.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "pisa.h"
+#include "pisa_internal.h"
+
+namespace pisa {
+
+static thread_local int32_t g_launches = 0;
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pisa_status make_plan(const pisa_shape* s, Plan* p) {
+    if (s == nullptr || p == nullptr) return PISA_ERR_INVALID_ARG;
+    memset(p, 0, sizeof(*p));
+    if (s->batch < 1 || s->heads_q < 1 || s->heads_kv < 1 || s->seq_q < 1 || s->seq_kv < 1 || s->head_dim < 1 ||
+        s->block < 1 || s->factor < 2 || s->topk < 1 || (s->causal != 0 && s->causal != 1) ||
+        (s->select_per_qhead != 0 && s->select_per_qhead != 1) || !(s->scale == s->scale))
+        return PISA_ERR_INVALID_ARG;
+    if (s->heads_q % s->heads_kv != 0) return PISA_ERR_INVALID_ARG;
+    if (s->seq_kv % s->block != 0) return PISA_ERR_INVALID_ARG;
+    if (s->seq_q != s->seq_kv && s->seq_q != 1) return PISA_ERR_INVALID_ARG;
+    if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
+    if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
+    // every row index must fit the 32-bit TMA coordinate and grid limits
+    const int64_t qrows = static_cast<int64_t>(s->batch) * s->heads_q * s->seq_q;
+    const int64_t krows = static_cast<int64_t>(s->batch) * s->heads_kv * s->seq_kv;
+    if (qrows >= (int64_t(1) << 31) || krows >= (int64_t(1) << 31)) return PISA_ERR_UNSUPPORTED;
+    if (s->batch > 65535) return PISA_ERR_UNSUPPORTED;
+
+    p->B = s->batch;
+    p->Hq = s->heads_q;
+    p->Hkv = s->heads_kv;
+    p->g = s->heads_q / s->heads_kv;
+    p->Nq = s->seq_q;
+    p->N = s->seq_kv;
+    p->D = s->head_dim;
+    p->blk = s->block;
+    p->f = s->factor;
+    p->topk = s->topk;
+    p->decode = s->seq_q == 1 ? 1 : 0;
+    p->causal = p->decode ? 0 : s->causal;
+    p->per_qhead = s->select_per_qhead;
+    p->scale = s->scale > 0.f ? s->scale : 1.0f / sqrtf(static_cast<float>(s->head_dim));
+    p->n0 = s->seq_kv / s->block;
+
+    int n = p->n0, L = 0, off = 0;
+    while (true) {
+        if (L >= PISA_MAX_LEVELS) return PISA_ERR_UNSUPPORTED;
+        p->lsize[L] = n;
+        p->loff[L] = off;
+        off += n;
+        ++L;
+        if (n <= p->f) break;
+        n = (n + p->f - 1) / p->f;
+    }
+    p->L = L;
+    p->total_nodes = off;
+    if (static_cast<int64_t>(p->f) * p->topk > PISA_MAX_CANDIDATES) return PISA_ERR_UNSUPPORTED;
+
+    p->Hsel = p->per_qhead ? p->Hq : p->Hkv;
+    p->gsel = p->per_qhead ? 1 : p->g;
+    p->nqb = p->decode ? 1 : p->Nq / p->blk;
+    if (p->Hsel > 65535 / 16) return PISA_ERR_UNSUPPORTED;
+    if (p->decode && p->gsel > 8) return PISA_ERR_UNSUPPORTED;
+
+    p->dec_bps = 4;
+    p->dec_splits = p->decode ? (p->topk + p->dec_bps - 1) / p->dec_bps : 0;
+
+    p->pyramid_bytes = static_cast<size_t>(p->B) * p->Hkv * p->total_nodes * p->D * sizeof(float);
+    size_t o = kStatusBytes;
+    p->ws_pyramid = o;
+    o = align256(o + p->pyramid_bytes);
+    p->ws_qbar = o;
+    o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->nqb * p->D * sizeof(float));
+    p->ws_idx = o;
+    o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->nqb * p->topk * sizeof(int32_t));
+    p->ws_part = o;
+    if (p->decode)
+        o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->dec_splits * p->gsel * (p->D + 2) * sizeof(float));
+    p->ws_total = o;
+    return PISA_OK;
+}
+
+// Heads of one attention CTA: the largest divisor of the shared group whose
+// rows fit two 128-row tensor-core tiles (one tile for 128-key blocks, whose
+// score tiles double the TMEM need).
+static int heads_per_cta(const Plan& pl) {
+    if (pl.per_qhead) return 1;
+    const int max_rows = pl.blk == 128 ? 128 : 256;
+    int best = 1;
+    for (int d = 1; d <= pl.g; ++d)
+        if (pl.g % d == 0 && d * pl.blk <= max_rows) best = d;
+    return best;
+}
+
+static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cudaStream_t st) {
+    MeanParams m{};
+    m.src = static_cast<const __nv_bfloat16*>(K);
+    m.dst = pyr;
+    m.Hsrc = pl.Hkv;
+    m.Nsrc = pl.N;
+    m.D = pl.D;
+    m.Hout = pl.Hkv;
+    m.rows_out = pl.n0;
+    m.dst_plane_rows = pl.total_nodes;
+    m.rows_per_group = pl.blk;
+    m.planes_per_group = 1;
+    m.batch = pl.B;
+    if (!launch_block_mean(m, st)) return PISA_ERR_CUDA;
+    ++g_launches;
+    int64_t width = 1;
+    for (int l = 1; l < pl.L; ++l) {
+        LevelParams lp{};
+        lp.pyr = pyr;
+        lp.planes = pl.B * pl.Hkv;
+        lp.plane_rows = pl.total_nodes;
+        lp.off_below = pl.loff[l - 1];
+        lp.off_cur = pl.loff[l];
+        lp.n_below = pl.lsize[l - 1];
+        lp.n_cur = pl.lsize[l];
+        lp.n0 = pl.n0;
+        lp.factor = pl.f;
+        lp.D = pl.D;
+        lp.width_below = width;
+        if (!launch_pyramid_level(lp, st)) return PISA_ERR_CUDA;
+        ++g_launches;
+        width *= pl.f;
+    }
+    return PISA_OK;
+}
+
+static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cudaStream_t st) {
+    MeanParams m{};
+    m.src = static_cast<const __nv_bfloat16*>(Q);
+    m.dst = qbar;
+    m.Hsrc = pl.Hq;
+    m.Nsrc = pl.Nq;
+    m.D = pl.D;
+    m.Hout = pl.Hsel;
+    m.rows_out = pl.nqb;
+    m.dst_plane_rows = pl.nqb;
+    m.rows_per_group = pl.decode ? 1 : pl.blk;
+    m.planes_per_group = pl.gsel;
+    m.batch = pl.B;
+    if (!launch_block_mean(m, st)) return PISA_ERR_CUDA;
+    ++g_launches;
+    return PISA_OK;
+}
+
+static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, const int32_t* budget,
+                          int32_t* idx, float* margin, uint32_t* status, cudaStream_t st) {
+    SelectParams sp{};
+    sp.qbar = qbar;
+    sp.pyr = pyr;
+    sp.idx = idx;
+    sp.margin = margin;
+    sp.status = status;
+    sp.Hsel = pl.Hsel;
+    sp.Hkv = pl.Hkv;
+    sp.gsel_div = pl.per_qhead ? pl.g : 1;
+    sp.nqb = pl.nqb;
+    sp.D = pl.D;
+    sp.n0 = pl.n0;
+    sp.factor = pl.f;
+    sp.topk = pl.topk;
+    sp.causal = pl.causal;
+    sp.decode = pl.decode;
+    sp.L = pl.L;
+    sp.total_nodes = pl.total_nodes;
+    int64_t w = 1;
+    for (int l = 0; l < pl.L; ++l) {
+        sp.lsize[l] = pl.lsize[l];
+        sp.loff[l] = pl.loff[l];
+        sp.budget[l] = budget ? budget[l] : pl.topk;
+        sp.width[l] = w;
+        w = w > (int64_t(1) << 40) ? w : w * pl.f;
+    }
+    if (!launch_select(sp, pl.B, st)) return PISA_ERR_CUDA;
+    ++g_launches;
+    return PISA_OK;
+}
+
+static pisa_status attention(const Plan& pl, const void* Q, const void* K, const void* V, const int32_t* idx,
+                             void* O, float* lse, uint8_t* ws, cudaStream_t st) {
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+    const float scale_log2 = pl.scale * 1.4426950408889634f;
+    if (pl.decode) {
+        DecodeParams d{};
+        d.Q = static_cast<const __nv_bfloat16*>(Q);
+        d.K = static_cast<const __nv_bfloat16*>(K);
+        d.V = static_cast<const __nv_bfloat16*>(V);
+        d.idx = idx;
+        d.part = reinterpret_cast<float*>(ws + pl.ws_part);
+        d.O = static_cast<__nv_bfloat16*>(O);
+        d.lse = lse;
+        d.status = status;
+        d.Hq = pl.Hq;
+        d.Hkv = pl.Hkv;
+        d.g = pl.g;
+        d.N = pl.N;
+        d.n0 = pl.n0;
+        d.D = pl.D;
+        d.blk = pl.blk;
+        d.topk = pl.topk;
+        d.per_qhead = pl.per_qhead;
+        d.Hsel = pl.Hsel;
+        d.gh = pl.gsel;
+        d.bps = pl.dec_bps;
+        d.splits = pl.dec_splits;
+        d.scale_log2 = scale_log2;
+        return launch_attn_decode(pl, d, st, &g_launches) ? PISA_OK : PISA_ERR_CUDA;
+    }
+    AttnParams a{};
+    a.idx = idx;
+    a.O = static_cast<__nv_bfloat16*>(O);
+    a.lse = lse;
+    a.status = status;
+    a.Hq = pl.Hq;
+    a.Hkv = pl.Hkv;
+    a.g = pl.g;
+    a.N = pl.N;
+    a.n0 = pl.n0;
+    a.topk = pl.topk;
+    a.causal = pl.causal;
+    a.per_qhead = pl.per_qhead;
+    a.Hsel = pl.Hsel;
+    a.nqb = pl.nqb;
+    a.gh = heads_per_cta(pl);
+    a.chunks = pl.per_qhead ? 1 : pl.g / a.gh;
+    a.scale_log2 = scale_log2;
+    return launch_attn_prefill(pl, Q, K, V, a, st, &g_launches);
+}
+
+static pisa_status check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
+    if (ws == nullptr || !aligned16(ws)) return PISA_ERR_INVALID_ARG;
+    if (ws_bytes < pl.ws_total) return PISA_ERR_WORKSPACE;
+    return PISA_OK;
+}
+
+}  // namespace pisa
+
+using namespace pisa;
+
+extern "C" {
+
+int32_t pisa_num_levels(const pisa_shape* shape) {
+    Plan pl;
+    return make_plan(shape, &pl) == PISA_OK ? pl.L : -1;
+}
+
+pisa_status pisa_level_layout(const pisa_shape* shape, int32_t* sizes, int32_t* offsets) {
+    Plan pl;
+    if (sizes == nullptr || offsets == nullptr) return PISA_ERR_INVALID_ARG;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    for (int l = 0; l < PISA_MAX_LEVELS; ++l) {
+        sizes[l] = l < pl.L ? pl.lsize[l] : 0;
+        offsets[l] = l < pl.L ? pl.loff[l] : 0;
+    }
+    return PISA_OK;
+}
+
+pisa_status pisa_pyramid_size(const pisa_shape* shape, size_t* bytes) {
+    Plan pl;
+    if (bytes == nullptr) return PISA_ERR_INVALID_ARG;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s == PISA_OK) *bytes = pl.pyramid_bytes;
+    return s;
+}
+
+pisa_status pisa_workspace_size(const pisa_shape* shape, size_t* bytes) {
+    Plan pl;
+    if (bytes == nullptr) return PISA_ERR_INVALID_ARG;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s == PISA_OK) *bytes = pl.ws_total;
+    return s;
+}
+
+pisa_status pisa_build_pyramid(const pisa_shape* shape, const void* K, float* pyramid, pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (K == nullptr || pyramid == nullptr || !aligned16(K) || !aligned16(pyramid)) return PISA_ERR_INVALID_ARG;
+    return build_pyramid(pl, K, pyramid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static pisa_status check_budget(const Plan& pl, const int32_t* level_budget) {
+    if (level_budget == nullptr) return PISA_OK;
+    if (level_budget[0] != pl.topk) return PISA_ERR_INVALID_ARG;
+    for (int l = 0; l < pl.L; ++l) {
+        if (level_budget[l] < 1) return PISA_ERR_INVALID_ARG;
+        if (static_cast<int64_t>(level_budget[l]) * pl.f > PISA_MAX_CANDIDATES) return PISA_ERR_UNSUPPORTED;
+    }
+    return PISA_OK;
+}
+
+pisa_status pisa_select_blocks(const pisa_shape* shape, const void* Q, const float* pyramid,
+                               const int32_t* level_budget, int32_t* idx, float* margin, void* ws, size_t ws_bytes,
+                               pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (Q == nullptr || pyramid == nullptr || idx == nullptr || !aligned16(Q) || !aligned16(pyramid) ||
+        !aligned16(idx))
+        return PISA_ERR_INVALID_ARG;
+    if ((s = check_budget(pl, level_budget)) != PISA_OK) return s;
+    if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
+    if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
+    return select(pl, qbar, pyramid, level_budget, idx, margin, reinterpret_cast<uint32_t*>(w), st);
+}
+
+pisa_status pisa_sparse_attention(const pisa_shape* shape, const void* Q, const void* K, const void* V,
+                                  const int32_t* idx, void* O, float* lse, void* ws, size_t ws_bytes,
+                                  pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (Q == nullptr || K == nullptr || V == nullptr || idx == nullptr || O == nullptr || !aligned16(Q) ||
+        !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx))
+        return PISA_ERR_INVALID_ARG;
+    if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    return attention(pl, Q, K, V, idx, O, lse, static_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+pisa_status pisa_forward(const pisa_shape* shape, const void* Q, const void* K, const void* V, void* O, float* lse,
+                         int32_t* idx_out, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr || !aligned16(Q) || !aligned16(K) ||
+        !aligned16(V) || !aligned16(O) || (idx_out != nullptr && !aligned16(idx_out)))
+        return PISA_ERR_INVALID_ARG;
+    if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float* pyr = reinterpret_cast<float*>(w + pl.ws_pyramid);
+    float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + pl.ws_idx);
+    if ((s = build_pyramid(pl, K, pyr, st)) != PISA_OK) return s;
+    if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
+    if ((s = select(pl, qbar, pyr, nullptr, idx, nullptr, reinterpret_cast<uint32_t*>(w), st)) != PISA_OK) return s;
+    return attention(pl, Q, K, V, idx, O, lse, w, st);
+}
+
+pisa_status pisa_check_status(void* ws, uint32_t* detail, pisa_stream_t stream) {
+    if (ws == nullptr) return PISA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t host[2] = {0, 0};
+    if (cudaMemcpyAsync(host, ws, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess) return PISA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+    if (host[0] != 0) {
+        if (cudaMemsetAsync(ws, 0, sizeof(host), st) != cudaSuccess) return PISA_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+    }
+    if (detail) *detail = host[1];
+    return static_cast<pisa_status>(host[0]);
+}
+
+const char* pisa_status_string(pisa_status status) {
+    switch (status) {
+        case PISA_OK: return "ok";
+        case PISA_ERR_INVALID_ARG: return "invalid argument";
+        case PISA_ERR_UNSUPPORTED: return "unsupported shape";
+        case PISA_ERR_WORKSPACE: return "workspace too small";
+        case PISA_ERR_CUDA: return "CUDA error";
+        case PISA_ERR_TIMEOUT: return "device wait timed out";
+        case PISA_ERR_BAD_INDEX: return "selected block index out of range";
+    }
+    return "unknown status";
+}
+
+int32_t pisa_last_launch_count(void) { return g_launches; }
+
+}  // extern "C"

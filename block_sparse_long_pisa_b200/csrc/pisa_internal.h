@@ -1,0 +1,120 @@
+// Internal definitions shared by the host-side API and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pisa.h"
+
+namespace pisa {
+
+// Upper bound on any single pipeline wait inside a kernel (ns).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bytes reserved for the status word at the start of the workspace.
+constexpr size_t kStatusBytes = 256;
+
+// Wait-site codes reported through the status word's detail field:
+// (kernel id << 8) | site.
+enum : uint32_t {
+    kKernAttnPrefill = 1,
+    kKernAttnDecode = 2,
+    kKernSelect = 3,
+};
+
+// Derived sizes of one problem (host side).
+struct Plan {
+    int32_t B, Hq, Hkv, g, Nq, N, D, blk, f, topk, causal, per_qhead, decode;
+    float scale;
+    int32_t n0;          // key blocks per sequence
+    int32_t L;           // pyramid levels
+    int32_t lsize[PISA_MAX_LEVELS];
+    int32_t loff[PISA_MAX_LEVELS];
+    int32_t total_nodes; // sum of level sizes (rows of one pyramid plane)
+    int32_t Hsel;        // selection rows per batch: Hkv (shared) or Hq (per query head)
+    int32_t nqb;         // query blocks: Nq / blk (prefill) or 1 (decode)
+    int32_t gsel;        // query heads averaged into one selection summary
+    // decode split-KV
+    int32_t dec_bps;     // selected blocks per split
+    int32_t dec_splits;
+    // workspace layout (byte offsets)
+    size_t ws_pyramid, ws_qbar, ws_idx, ws_part, ws_total;
+    size_t pyramid_bytes;
+};
+
+// Validates a shape and fills the plan. Host only, never touches the GPU.
+pisa_status make_plan(const pisa_shape* s, Plan* p);
+
+// ---------------------------------------------------------------- kernel parameter blocks
+
+struct MeanParams {
+    const __nv_bfloat16* src;   // bf16 [.., Hsrc, Nsrc, D]
+    float* dst;                 // fp32 rows
+    int32_t Hsrc, Nsrc, D;
+    int32_t Hout;               // output planes per batch
+    int32_t rows_out;           // output rows per plane (n0 or nqb)
+    int32_t dst_plane_rows;     // row stride between output planes
+    int32_t rows_per_group;     // source rows averaged per output row (block, or 1)
+    int32_t planes_per_group;   // consecutive source heads averaged (g or 1)
+    int32_t batch;
+};
+
+struct LevelParams {
+    float* pyr;                 // pyramid base
+    int32_t planes;             // batch * heads_kv
+    int32_t plane_rows;         // total_nodes
+    int32_t off_below, off_cur; // row offsets of the two levels inside a plane
+    int32_t n_below, n_cur;
+    int32_t n0, factor, D;
+    int64_t width_below;        // level-0 blocks under one node of the level below (f^(l-1))
+};
+
+struct SelectParams {
+    const float* qbar;          // fp32 [B, Hsel, nqb, D]
+    const float* pyr;           // fp32 [B, Hkv, total_nodes, D]
+    int32_t* idx;               // int32 [B, Hsel, nqb, topk]
+    float* margin;              // optional fp32 [B, Hsel, nqb]
+    uint32_t* status;
+    int32_t Hsel, Hkv, gsel_div, nqb, D, n0, factor, topk, causal, decode, L, total_nodes;
+    int32_t lsize[PISA_MAX_LEVELS];
+    int32_t loff[PISA_MAX_LEVELS];
+    int32_t budget[PISA_MAX_LEVELS];
+    int64_t width[PISA_MAX_LEVELS];  // f^l (saturated)
+};
+
+struct AttnParams {
+    const int32_t* idx;         // [B, Hsel, nqb, topk]
+    __nv_bfloat16* O;           // [B, Hq, N, D]
+    float* lse;                 // optional [B, Hq, N]
+    uint32_t* status;
+    int32_t Hq, Hkv, g, N, n0, topk, causal, per_qhead, Hsel, nqb;
+    int32_t gh;                 // query heads in one CTA
+    int32_t chunks;             // CTAs per (batch, selection row, query block) = heads / gh
+    float scale_log2;           // softmax scale * log2(e)
+};
+
+struct DecodeParams {
+    const __nv_bfloat16* Q;     // [B, Hq, 1, D]
+    const __nv_bfloat16* K;     // [B, Hkv, N, D]
+    const __nv_bfloat16* V;
+    const int32_t* idx;         // [B, Hsel, 1, topk]
+    float* part;                // [B, Hsel, splits, gh, D + 2]
+    __nv_bfloat16* O;           // [B, Hq, 1, D]
+    float* lse;                 // optional [B, Hq, 1]
+    uint32_t* status;
+    int32_t Hq, Hkv, g, N, n0, D, blk, topk, per_qhead, Hsel, gh, bps, splits;
+    float scale_log2;
+};
+
+// ---------------------------------------------------------------- launchers (return false on launch error)
+
+bool launch_block_mean(const MeanParams& p, cudaStream_t st);
+bool launch_pyramid_level(const LevelParams& p, cudaStream_t st);
+bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st);
+// Prefill attention: builds the tensor maps and picks the kernel variant.
+pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
+                                cudaStream_t st, int32_t* launches);
+bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
+
+}  // namespace pisa

@@ -1,0 +1,180 @@
+/*
+ * pisa.h - C ABI of the B200 (sm_100a) PISA pyramid block-sparse attention library.
+ *
+ * The method, as described in "Attention clairsemee PISA : noyaux Triton sans
+ * matrice de scores" (irisproject.cloud):
+ *   1. keys are mean-pooled into blocks, then into coarser and coarser levels
+ *      (sections "Une pyramide de cles plutot qu'un tapis uniforme" and
+ *      "Le pooling comme premiere reduction");
+ *   2. each query block descends that pyramid, keeping its top-K blocks
+ *      (section "La selection top-K guidee par la pyramide");
+ *   3. exact softmax attention runs over the selected key/value blocks only,
+ *      fused so that no score matrix is written to memory (section
+ *      "Des noyaux Triton qui ne materialisent rien").
+ *
+ * Conventions shared by every call:
+ *   - Q, K, V, O are bf16, contiguous [batch, heads, tokens, head_dim] with
+ *     head_dim innermost. Device pointers, 16-byte aligned.
+ *   - The caller owns and allocates every buffer, the workspace included.
+ *     The library never allocates or frees memory and never synchronises,
+ *     except pisa_check_status, which synchronises the given stream.
+ *   - Every compute call only enqueues work on `stream` and returns.
+ *   - Argument errors are detected on the host, before anything is enqueued,
+ *     and returned synchronously. A failed kernel launch returns
+ *     PISA_ERR_CUDA. Errors a kernel detects on the device (an index outside
+ *     the eligible blocks, a pipeline wait that ran out of time) are recorded
+ *     in the status word at the start of the workspace and reported by
+ *     pisa_check_status; the kernel skips the offending work and returns.
+ *   - Argument checks never touch the GPU, so they can be exercised on a host
+ *     without one.
+ */
+#ifndef PISA_H
+#define PISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PISA_API __attribute__((visibility("default")))
+#else
+#define PISA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). NULL is the legacy default stream. */
+typedef struct CUstream_st *pisa_stream_t;
+
+/* Problem description shared by every call.
+ *   batch, heads_q, heads_kv : heads_q % heads_kv == 0 (g = heads_q / heads_kv query
+ *                              heads share one KV head; g = 1 is multi-head attention).
+ *   seq_kv                   : keys per sequence, a multiple of `block`.
+ *   seq_q                    : == seq_kv for prefill (query t sits at position t);
+ *                              == 1 for decode (the query sits at position seq_kv - 1).
+ *   head_dim                 : 64 or 128.
+ *   block                    : key-block size b (and query-block size for prefill): 64 or 128.
+ *   factor                   : pooling factor f >= 2 between pyramid levels.
+ *   topk                     : K, key blocks kept per query block, 1 <= K.
+ *   causal                   : 0/1. Prefill only: query block i may use key blocks j <= i
+ *                              and, inside block i, keys at or before the query.
+ *   select_per_qhead         : 0 = one selection per (batch, KV head, query block) from the
+ *                              mean over the g query heads (default); 1 = one selection per
+ *                              query head.
+ *   scale                    : softmax scale; <= 0 selects 1/sqrt(head_dim). */
+typedef struct {
+    int32_t batch, heads_q, heads_kv, seq_q, seq_kv, head_dim;
+    int32_t block, factor, topk, causal;
+    int32_t select_per_qhead;
+    float scale;
+} pisa_shape;
+
+typedef enum {
+    PISA_OK = 0,
+    PISA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent shape                */
+    PISA_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for                 */
+    PISA_ERR_WORKSPACE = 3,    /* workspace smaller than pisa_workspace_size                 */
+    PISA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed                        */
+    PISA_ERR_TIMEOUT = 5,      /* device: a pipeline wait ran out of time                    */
+    PISA_ERR_BAD_INDEX = 6     /* device: a selected block outside [0, n0) or after the query */
+} pisa_status;
+
+#define PISA_MAX_LEVELS 24
+/* Largest candidate set one pyramid level may score: factor * max level budget. */
+#define PISA_MAX_CANDIDATES 4096
+
+/* Number of pyramid levels L (n_0 = seq_kv / block, n_{l+1} = ceil(n_l / factor),
+ * built while n_l > factor), or -1 if the shape is invalid. Host only. */
+PISA_API int32_t pisa_num_levels(const pisa_shape *shape);
+
+/* Node count n_l and row offset of every level inside one (batch, KV head) plane
+ * of the pyramid buffer. `sizes` and `offsets` hold at least PISA_MAX_LEVELS
+ * entries; unused entries are set to 0. Host only. */
+PISA_API pisa_status pisa_level_layout(const pisa_shape *shape, int32_t *sizes, int32_t *offsets);
+
+/* Bytes of the pyramid buffer: fp32 [batch, heads_kv, sum_l n_l, head_dim].
+ * Level l of plane (b, h) starts at row offsets[l] of that plane. Host only. */
+PISA_API pisa_status pisa_pyramid_size(const pisa_shape *shape, size_t *bytes);
+
+/* Bytes of workspace that pisa_forward, pisa_select_blocks and
+ * pisa_sparse_attention need for this shape (one size serves all three).
+ * The first 256 bytes are the device status word; zero them once when the
+ * workspace is allocated (pisa_check_status clears them after each read).
+ * Host only. */
+PISA_API pisa_status pisa_workspace_size(const pisa_shape *shape, size_t *bytes);
+
+/* Step 1, the key pyramid ("Le pooling comme premiere reduction"): level 0 is
+ * the fp32 mean of every key block of `block` keys; a node of level l+1 is the
+ * mean of its children weighted by the level-0 blocks each covers (so every
+ * node is the mean of all keys under it).
+ *   K        : bf16 [batch, heads_kv, seq_kv, head_dim], device.
+ *   pyramid  : fp32 output, pisa_pyramid_size bytes, device. */
+PISA_API pisa_status pisa_build_pyramid(const pisa_shape *shape, const void *K, float *pyramid,
+                               pisa_stream_t stream);
+
+/* Step 2, pyramid-guided top-K ("La selection top-K guidee par la pyramide").
+ * For every query block: its summary q = mean of its queries (over the g query
+ * heads of the KV head unless select_per_qhead; decode: the single token);
+ * start from every eligible node of the top level; at each level score the
+ * candidates by the fp32 dot product q . node, keep the best K_l (higher score
+ * first, lower node index on equal scores; all of them if there are no more
+ * than K_l) and descend to their children. Causal: only blocks j <= i are
+ * eligible and a node that straddles block i is scored with the mean of its
+ * eligible blocks.
+ *   Q            : bf16 queries (layout above), device.
+ *   pyramid      : fp32 pyramid from pisa_build_pyramid, device.
+ *   level_budget : HOST array of L budgets K_l (level 0 first, K_0 == topk), or
+ *                  NULL for K at every level.
+ *   idx          : int32 output [batch, Hsel, nQB, topk], device; Hsel = heads_kv
+ *                  (shared) or heads_q (per query head); nQB = seq_q / block
+ *                  (prefill) or 1 (decode). Each row lists the kept blocks in
+ *                  ascending order, padded with -1.
+ *   margin       : optional fp32 output [batch, Hsel, nQB], device: smallest
+ *                  relative gap (s_K - s_K+1) / max(|s_K|, |s_K+1|) met at a
+ *                  pruning level (+inf if no level was pruned). NULL to skip.
+ *   ws, ws_bytes : workspace (pisa_workspace_size), device. */
+PISA_API pisa_status pisa_select_blocks(const pisa_shape *shape, const void *Q, const float *pyramid,
+                               const int32_t *level_budget, int32_t *idx, float *margin,
+                               void *ws, size_t ws_bytes, pisa_stream_t stream);
+
+/* Step 3, fused block-sparse attention ("Des noyaux Triton qui ne
+ * materialisent rien"): for every query row, S = scale * q . k over the keys
+ * of the blocks listed in its idx row (keys after the query masked when
+ * causal), O = softmax(S) V and LSE = log sum exp S, computed tile by tile
+ * with an online softmax; scores never leave on-chip memory.
+ *   idx   : int32 [batch, Hsel, nQB, topk] as produced by pisa_select_blocks;
+ *           entries < 0 are skipped; an entry >= n0, or > i when causal,
+ *           is skipped and recorded as PISA_ERR_BAD_INDEX. Entries must be
+ *           distinct (a repeated block is attended twice).
+ *   O     : bf16 output, same layout as Q, device.
+ *   lse   : optional fp32 output [batch, heads_q, seq_q] (natural log), or NULL.
+ * A query row whose idx row holds no valid block gets O = 0 and LSE = -inf. */
+PISA_API pisa_status pisa_sparse_attention(const pisa_shape *shape, const void *Q, const void *K,
+                                  const void *V, const int32_t *idx, void *O, float *lse,
+                                  void *ws, size_t ws_bytes, pisa_stream_t stream);
+
+/* Steps 1-3 in one call on one stream: pyramid and query summaries into the
+ * workspace, selection, attention.
+ *   idx_out : optional int32 [batch, Hsel, nQB, topk] copy of the selection
+ *             (NULL keeps it in the workspace). */
+PISA_API pisa_status pisa_forward(const pisa_shape *shape, const void *Q, const void *K, const void *V,
+                         void *O, float *lse, int32_t *idx_out, void *ws, size_t ws_bytes,
+                         pisa_stream_t stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded in the
+ * workspace status word since the last call (PISA_OK if none) and clears it.
+ * `detail`, if not NULL, receives a code locating the error (kernel and wait site). */
+PISA_API pisa_status pisa_check_status(void *ws, uint32_t *detail, pisa_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+PISA_API const char *pisa_status_string(pisa_status status);
+
+/* Kernel launches the last compute call on this host thread enqueued. */
+PISA_API int32_t pisa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H */

@@ -182,8 +182,12 @@ def attend(q_rows: np.ndarray, q_pos: np.ndarray, k_plane: np.ndarray, v_plane: 
 
     S = scale * q . k for every key of every selected block, keys after the
     query position masked when causal; O = softmax(S) V; LSE = log sum exp S.
-    Returns O [R, D] and LSE [R].
+    Returns O [R, D] and LSE [R]. A row with no selected block has no key to
+    attend to: O = 0 and LSE = -inf (the library's convention for that case).
     """
+    if len(blocks) == 0:
+        return (np.zeros((q_rows.shape[0], v_plane.shape[1]), dtype=F32),
+                np.full(q_rows.shape[0], -np.inf, dtype=F32))
     key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
     kx = k_plane[key_pos].astype(F32)
     vx = v_plane[key_pos].astype(F32)

@@ -1,0 +1,48 @@
+"""Helpers for the GPU parity tests: seeded inputs on the device, oracle
+references on the host, and the acceptance checks.
+
+Acceptance (bf16 inputs, fp32 accumulation):
+  * selected indices bit-exact, except query blocks whose oracle margin at a
+    pruning level is below 1e-3 (near-ties), which are counted;
+  * O within max-abs 2e-2 and mean-abs 2e-3 of the oracle run on the GPU's own
+    indices; LSE within 1e-3;
+  * pyramid within 1e-5 absolute + 1e-5 relative.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import workloads
+
+O_MAX, O_MEAN, LSE_TOL, PYR_TOL, NEAR_TIE = 2e-2, 2e-3, 1e-3, 1e-5, 1e-3
+
+
+to_device = workloads.device_tensor
+
+
+def host_f32(t):
+    """fp32 numpy copy of a bf16/fp32 device tensor."""
+    return t.float().cpu().numpy()
+
+
+def selection_report(gpu_idx, ref_idx, ref_margin):
+    """(mismatching rows that are not near-ties, near-tie rows) over rows given as arrays [..., K]."""
+    same = np.all(gpu_idx == ref_idx, axis=-1)
+    near = np.asarray(ref_margin) < NEAR_TIE
+    return int(np.sum(~same & ~near)), int(np.sum(near))
+
+
+def assert_output_close(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
+    err = np.abs(np.asarray(o_gpu, dtype=np.float64) - np.asarray(o_ref, dtype=np.float64))
+    assert err.max() < O_MAX, f"{what}: O max-abs {err.max():.3e}"
+    assert err.mean() < O_MEAN, f"{what}: O mean-abs {err.mean():.3e}"
+    if lse_gpu is not None:
+        le = np.abs(np.asarray(lse_gpu, dtype=np.float64) - np.asarray(lse_ref, dtype=np.float64))
+        assert le.max() < LSE_TOL, f"{what}: LSE max-abs {le.max():.3e}"
+
+
+def assert_pyramid_close(pyr_gpu, levels_ref, offsets):
+    for l, lev in enumerate(levels_ref):
+        got = pyr_gpu[offsets[l]:offsets[l] + lev.shape[0]]
+        err = np.abs(got - lev)
+        assert np.all(err <= PYR_TOL + PYR_TOL * np.abs(lev)), f"level {l}: max err {err.max():.3e}"

@@ -1,0 +1,231 @@
+"""GPU path vs the CPU oracle on seeded inputs, through the C ABI.
+
+Small shapes: every kernel variant (head dims 64/128, blocks 64/128, 1 or 2
+tensor-core tiles per CTA, split head groups), causal and not, shared and
+per-query-head selection, ragged pyramids, decode, ties and edge cases.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+W = workloads.Workload
+
+SMALL = {
+    "tiny": workloads.WORKLOADS["tiny"],
+    "gqa4-causal-ragged": W("gqa4-causal-ragged", 1, 8, 2, 37 * 64, 37 * 64, 128, 64, 4, 6, 1, "iid", 11),
+    "gqa2-causal": W("gqa2-causal", 1, 4, 2, 20 * 64, 20 * 64, 128, 64, 4, 5, 1, "iid", 12),
+    "gqa8-d64-causal": W("gqa8-d64-causal", 1, 16, 2, 24 * 64, 24 * 64, 64, 64, 4, 4, 1, "iid", 13),
+    "mha-d128-b64-causal": W("mha-d128-b64-causal", 1, 3, 3, 33 * 64, 33 * 64, 128, 64, 4, 7, 1, "clustered", 14),
+    "mha-d64-b128-f8": W("mha-d64-b128-f8", 1, 2, 2, 70 * 128, 70 * 128, 64, 128, 8, 9, 0, "iid", 15),
+    "mha-d128-b128-f8-causal": W("mha-d128-b128-f8-causal", 1, 2, 2, 66 * 128, 66 * 128, 128, 128, 8, 10, 1,
+                                 "clustered", 16),
+    "gqa4-d64-noncausal": W("gqa4-d64-noncausal", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 5, 0, "iid", 17),
+    "gqa4-needle": W("gqa4-needle", 1, 8, 2, 256 * 64, 256 * 64, 128, 64, 4, 16, 1, "needle", 18),
+    "decode-gqa4": W("decode-gqa4", 3, 8, 2, 1, 45 * 64, 128, 64, 4, 9, 0, "clustered", 19),
+    "decode-d64-b128": W("decode-d64-b128", 2, 4, 4, 1, 40 * 128, 64, 128, 8, 6, 0, "iid", 20),
+}
+PER_QHEAD = {
+    "perq-gqa4-causal": W("perq-gqa4-causal", 1, 8, 2, 21 * 64, 21 * 64, 128, 64, 4, 5, 1, "iid", 21),
+    "perq-decode": W("perq-decode", 2, 8, 2, 1, 30 * 64, 128, 64, 4, 7, 0, "iid", 22),
+}
+
+
+def _run(w, cuda_device, per_qhead=False, topk=None):
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    if topk is not None:
+        w = w.replace(topk=topk)
+    shape = pisa.Shape.of(w, select_per_qhead=int(per_qhead))
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    pyr = pisa.build_pyramid(shape, k)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, w.name)
+    assert pisa.last_launch_count() >= 1
+    Q, K, V = (gu.host_f32(x) for x in (q, k, v))
+    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_qhead)
+    return shape, (Q, K, V), ref, gu.host_f32(o), gu.host_f32(lse), idx.cpu().numpy(), gu.host_f32(pyr)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL) + sorted(PER_QHEAD))
+def test_forward_matches_oracle(name, cuda_device):
+    per_q = name in PER_QHEAD
+    w = PER_QHEAD[name] if per_q else SMALL[name]
+    shape, (Q, K, V), ref, o, lse, idx, pyr = _run(w, cuda_device, per_qhead=per_q)
+    import block_sparse_long_pisa_b200 as pisa
+    _, offs = pisa.level_layout(shape)
+    for b in range(w.batch):
+        for h in range(w.heads_kv):
+            gu.assert_pyramid_close(pyr[b, h], ref["pyramid"][b][h], offs)
+    bad, near = gu.selection_report(idx, ref["idx"], ref["margin"])
+    assert bad == 0, f"{bad} selections differ outside near-ties ({near} near-ties)"
+    # attention checked against the oracle on the GPU's own selection
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_q, idx_override=idx)
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"], name)
+    if w.keys == "needle":
+        for kvh in range(w.heads_kv):
+            for (i, j) in workloads.needles(w, 0, kvh):
+                assert j in idx[0, kvh, i], (kvh, i, j)
+
+
+@pytest.mark.parametrize("name", ["gqa4-causal-ragged", "mha-d64-b128-f8", "decode-gqa4"])
+def test_full_topk_is_dense_attention(name, cuda_device):
+    """K >= number of blocks: every eligible block is selected and O is dense softmax attention."""
+    w = SMALL[name]
+    n0 = w.n_blocks
+    shape, (Q, K, V), ref, o, lse, idx, _ = _run(w, cuda_device, topk=n0)
+    g = w.group
+    scale = 1.0 / math.sqrt(w.head_dim)
+    for b in range(w.batch):
+        for h in range(w.heads_q):
+            pos = np.full(1, w.seq_kv - 1) if w.decode else np.arange(w.seq_q)
+            d_o, d_l = oracle.dense_attention(Q[b, h], pos, K[b, h // g], V[b, h // g],
+                                              bool(w.causal) and not w.decode, scale)
+            gu.assert_output_close(o[b, h], d_o, lse[b, h], d_l, f"{name} b{b} h{h}")
+    if not w.decode:
+        nqb = w.seq_q // w.block
+        for i in range(nqb):
+            expect = list(range(i + 1)) if w.causal else list(range(n0))
+            assert idx[0, 0, i, :len(expect)].tolist() == expect
+            assert np.all(idx[0, 0, i, len(expect):] == -1)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_small_topk(topk, cuda_device):
+    w = SMALL["gqa4-causal-ragged"]
+    shape, (Q, K, V), ref, o, lse, idx, _ = _run(w, cuda_device, topk=topk)
+    bad, _ = gu.selection_report(idx, ref["idx"], ref["margin"])
+    assert bad == 0
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, topk, True, idx_override=idx)
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"])
+
+
+def _tie_inputs(device):
+    """Key blocks 3, 9 and 12 identical and aligned with every query; all others zero.
+
+    nb = 16, f = 4, K = 2: level-1 nodes 0, 2, 3 tie exactly; lower indices win
+    at every level, so every query block must select exactly [3, 9].
+    """
+    import torch
+    D, b, nb = 64, 64, 16
+    k = torch.zeros((1, 1, nb * b, D), dtype=torch.bfloat16)
+    pattern = torch.zeros(D)
+    pattern[0], pattern[1] = 1.0, 0.5
+    for j in (3, 9, 12):
+        k[0, 0, j * b:(j + 1) * b] = pattern
+    q = torch.zeros((1, 1, nb * b, D), dtype=torch.bfloat16)
+    q[..., 0] = 1.0
+    v = torch.randn((1, 1, nb * b, D), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    return [x.to(device) for x in (q, k, v)]
+
+
+def test_exact_ties_go_to_lower_index(cuda_device):
+    import block_sparse_long_pisa_b200 as pisa
+    q, k, v = _tie_inputs(cuda_device)
+    shape = pisa.Shape(1, 1, 1, 1024, 1024, 64, 64, 4, 2, causal=0)
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    pisa.raise_on_device_error(ws)
+    idx = idx.cpu().numpy()
+    assert np.all(idx[0, 0] == np.array([3, 9])), idx[0, 0]
+    ref = oracle.forward(*(gu.host_f32(x) for x in (q, k, v)), 64, 4, 2, False)
+    assert np.array_equal(idx, ref["idx"])
+
+
+def test_full_budgets_equal_exhaustive_topk(cuda_device):
+    """level_budget = n_l at every coarse level: the descent is exhaustive top-K."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL["gqa4-causal-ragged"]
+    shape = pisa.Shape.of(w)
+    q, k = (gu.to_device(w, t, cuda_device) for t in ("q", "k"))
+    sizes, _ = pisa.level_layout(shape)
+    budgets = [w.topk] + sizes[1:]
+    ws = pisa.new_workspace(shape, cuda_device)
+    pyr = pisa.build_pyramid(shape, k)
+    idx, marg = pisa.select_blocks(shape, q, pyr, ws, level_budget=budgets, margin=True)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws)
+    idx = idx.cpu().numpy()
+    Q, K = gu.host_f32(q), gu.host_f32(k)
+    for h in range(w.heads_kv):
+        qbar = oracle.query_summary(Q[0, h * w.group:(h + 1) * w.group], w.block)
+        for i in range(w.seq_q // w.block):
+            nb = i + 1
+            means = K[0, h].astype(np.float64).reshape(-1, w.block, w.head_dim).mean(1)[:nb]
+            s = means @ qbar[i].astype(np.float64)
+            order = sorted(range(nb), key=lambda j: (-s[j], j))
+            if nb > w.topk and (s[order[w.topk - 1]] - s[order[w.topk]]) < 1e-3 * abs(s[order[w.topk - 1]]):
+                continue
+            expect = sorted(order[:w.topk])
+            assert idx[0, h, i, :len(expect)].tolist() == expect, (h, i)
+
+
+def test_sparse_attention_on_given_indices_and_bad_entries(cuda_device):
+    """Arbitrary index rows: -1 padding is skipped, out-of-range or future blocks are skipped and reported,
+    and a row with no valid block gives O = 0 and LSE = -inf."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL["gqa2-causal"]
+    shape = pisa.Shape.of(w)
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    nqb, K = w.seq_q // w.block, w.topk
+    rng = np.random.Generator(np.random.PCG64(5))
+    idx = np.full((1, w.heads_kv, nqb, K), -1, dtype=np.int32)
+    for h in range(w.heads_kv):
+        for i in range(nqb):
+            n = int(rng.integers(1, min(K, i + 1) + 1))
+            idx[0, h, i, :n] = np.sort(rng.choice(i + 1, size=n, replace=False))
+    idx[0, 1, 4] = -1                       # empty row
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse = pisa.sparse_attention(shape, q, k, v, torch.from_numpy(idx).to(cuda_device), ws)
+    st, _ = pisa.check_status(ws)
+    assert st == pisa.OK
+    Q, Kf, V = (gu.host_f32(x) for x in (q, k, v))
+    ref = oracle.forward(Q, Kf, V, w.block, w.factor, K, True, idx_override=idx)
+    o, lse = gu.host_f32(o), gu.host_f32(lse)
+    g = w.group
+    rows = slice(4 * w.block, 5 * w.block)
+    assert np.all(o[0, g:2 * g, rows] == 0) and np.all(np.isneginf(lse[0, g:2 * g, rows]))
+    keep = np.ones(o.shape, dtype=bool)
+    keep[0, g:2 * g, rows] = False
+    gu.assert_output_close(o[keep], ref["O"][keep], what="given indices")
+    # a future block (causal) and an out-of-range block are skipped and reported
+    bad = idx.copy()
+    bad[0, 0, 2, -1] = 7                    # j > i for i = 2
+    bad[0, 0, 3, -1] = 10 ** 6              # j >= n0
+    o2, _ = pisa.sparse_attention(shape, q, k, v, torch.from_numpy(bad).to(cuda_device), ws)
+    st, _ = pisa.check_status(ws)
+    assert st == pisa.ERR_BAD_INDEX
+    o2 = gu.host_f32(o2)
+    np.testing.assert_array_equal(o2[0, :g, 2 * 64:4 * 64], o[0, :g, 2 * 64:4 * 64])
+    assert pisa.check_status(ws)[0] == pisa.OK  # cleared after the read
+
+
+def test_decode_split_merge_matches_unsplit(cuda_device):
+    """Many splits (K = 40 blocks -> 10 splits) merged by LSE equal the oracle's single softmax."""
+    w = W("decode-many-splits", 2, 4, 1, 1, 96 * 64, 128, 64, 4, 40, 0, "iid", 31)
+    shape, (Q, K, V), ref, o, lse, idx, _ = _run(w, cuda_device)
+    bad, _ = gu.selection_report(idx, ref["idx"], ref["margin"])
+    assert bad == 0
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, idx_override=idx)
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"])
+
+
+def test_repeated_calls_are_deterministic(cuda_device):
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL["gqa4-causal-ragged"]
+    shape = pisa.Shape.of(w)
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    o1, l1, i1 = pisa.forward(shape, q, k, v, ws, idx=True)
+    o2, l2, i2 = pisa.forward(shape, q, k, v, ws, idx=True)
+    pisa.raise_on_device_error(ws)
+    assert (i1 == i2).all() and (o1 == o2).all() and (l1 == l2).all()

@@ -228,3 +228,23 @@ def tensor_bf16(w: Workload, tensor: str, out: np.ndarray | None = None, threads
 def qkv_f32(w: Workload) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Small workloads only: Q, K, V as bf16-exact fp32 arrays [B, H, rows, D]."""
     return tuple(bf16_to_f32(tensor_bf16(w, t)) for t in ("q", "k", "v"))
+
+
+def device_tensor(w: Workload, tensor: str, device):
+    """bf16 torch tensor [B, H, rows, D] on `device`, drawn batch by batch (bounded host memory)."""
+    import torch
+    heads = w.heads_q if tensor == "q" else w.heads_kv
+    rows = _rows(w, tensor)
+    out = torch.empty((w.batch, heads, rows, w.head_dim), dtype=torch.bfloat16, device=device)
+    n_chunks = (rows + CHUNK_ROWS - 1) // CHUNK_ROWS
+    host = np.empty((heads, rows, w.head_dim), dtype=np.uint16)
+    threads = min(32, os.cpu_count() or 1)
+    for b in range(w.batch):
+        def run(job, b=b):
+            h, c = job
+            r0 = c * CHUNK_ROWS
+            host[h, r0:min(r0 + CHUNK_ROWS, rows)] = chunk_bf16(w, tensor, b, h, c)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(run, [(h, c) for h in range(heads) for c in range(n_chunks)]))
+        out[b].copy_(torch.from_numpy(host.view(np.int16)).view(torch.bfloat16))
+    return out
