@@ -47,15 +47,19 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profiled_traffic(kernel_file: str) -> float | None:
-    """dram bytes per launch recorded by an ncu capture summary (profiles/<file>), if present."""
+def profiled_traffic(kernel_file: str, source: str) -> float | None:
+    """dram bytes per launch recorded by an ncu capture summary (profiles/<file>), or None when
+    absent or when the kernel source has changed since the capture (sha256 prefix recorded there)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", kernel_file)
     if not os.path.exists(p):
         return None
-    for line in open(p):
-        if line.startswith("dram_bytes_per_launch_full_size:"):
-            return float(line.split(":", 1)[1].strip())
-    return None
+    sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    fields = dict(line.split(":", 1) for line in open(p) if ":" in line and not line.startswith((" ", "|", "#")))
+    if fields.get("source_sha256_16", "").strip() != sha:
+        return None
+    v = fields.get("dram_bytes_per_launch_full_size")
+    return float(v) if v is not None else None
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -103,7 +107,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -120,7 +124,7 @@ class ClockSampler:
         sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if len(r) >= 9 and r[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4) if "Active" in r[5 + i]})
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4) if r[5 + i].strip() == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": reasons, "samples": len(rows)}
 
@@ -228,7 +232,7 @@ def run_gpu(args, world, rank, local):
     import block_sparse_long_pisa_b200 as pisa
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = rank_workload(workloads.WORKLOADS[WORKLOAD], rank)
+    w = rank_workload(bench_workload(args), rank)
     shape = pisa.Shape.of(w)
     q, k, v = (workloads.device_tensor(w, t, dev) for t in ("q", "k", "v"))
     ws = pisa.new_workspace(shape, dev)
@@ -302,7 +306,7 @@ def run_gpu(args, world, rank, local):
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
-    if rank == 0:
+    if rank == 0 and not args.no_e2e:
         sess = pisa.Session(shape, dev)
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         hout = torch.empty(tuple(q.shape), dtype=torch.bfloat16).pin_memory()
@@ -325,8 +329,8 @@ def run_gpu(args, world, rank, local):
 
     if rank != 0:
         return
-    cpu = oracle_sample(workloads.WORKLOADS[WORKLOAD]) if world == 1 and not args.no_cpu_baseline else None
-    traffic = profiled_traffic("attn_prefill_gqa128k.md")
+    cpu = oracle_sample(bench_workload(args)) if world == 1 and not args.no_cpu_baseline else None
+    traffic = profiled_traffic("attn_prefill_gqa128k.md", "block_sparse_long_pisa_b200/csrc/attn_prefill.cu")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -347,6 +351,15 @@ def run_gpu(args, world, rank, local):
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def bench_workload(args):
+    w = workloads.WORKLOADS[args.workload]
+    if w.decode:
+        raise SystemExit("bench.py times prefill workloads; decode is covered by the parity tests")
+    if args.seq:
+        w = w.replace(seq_q=args.seq, seq_kv=args.seq, name=f"{w.name}@N={args.seq}")
+    return w
 
 
 def scored_candidates(shape, sizes) -> int:
@@ -371,6 +384,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS),
+                    help="prefill workload to time (default: the N=128K GQA workload)")
+    ap.add_argument("--seq", type=int, default=0, help="override the sequence length (smaller profiling cases)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.impl == "reference":

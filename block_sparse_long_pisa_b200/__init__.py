@@ -217,7 +217,7 @@ def sparse_attention(shape: Shape, Q, K, V, idx, ws, O=None, lse=True, stream=No
     _need(Q, torch.bfloat16, (B, Hq, Nq, D), "Q")
     if O is None:
         O = torch.empty_like(Q)
-    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else (lse or None)
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else lse
     _check(_lib.pisa_sparse_attention(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O),
                                       _ptr(L), _ptr(ws), ws.numel(), _stream(stream)), "pisa_sparse_attention")
     return O, L
@@ -232,7 +232,7 @@ def forward(shape: Shape, Q, K, V, ws, O=None, lse=True, idx=None, stream=None):
     _need(V, torch.bfloat16, (B, shape.heads_kv, shape.seq_kv, D), "V")
     if O is None:
         O = torch.empty_like(Q)
-    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else (lse or None)
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else lse
     if idx is True:
         idx = torch.empty((B, shape.hsel, shape.n_qblocks, shape.topk), dtype=torch.int32, device=Q.device)
     _check(_lib.pisa_forward(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(L), _ptr(idx),
