@@ -60,6 +60,7 @@ _sig = {
     "pisa_check_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
     "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pisa_last_launch_count": (ctypes.c_int32, []),
+    "pisa_decode_attention_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -238,6 +239,19 @@ def forward(shape: Shape, Q, K, V, ws, O=None, lse=True, idx=None, stream=None):
     _check(_lib.pisa_forward(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(L), _ptr(idx),
                              _ptr(ws), ws.numel(), _stream(stream)), "pisa_forward")
     return O, L, idx
+
+
+def decode_attention_noalloc(shape: Shape, Q, K, V, idx, O=None, lse=True, stream=None):
+    """Decode attention with the library's built-in scratch (no workspace, no allocation inside)."""
+    torch = _torch()
+    B, Hq, D = shape.batch, shape.heads_q, shape.head_dim
+    _need(Q, torch.bfloat16, (B, Hq, 1, D), "Q")
+    if O is None:
+        O = torch.empty_like(Q)
+    L = torch.empty((B, Hq, 1), dtype=torch.float32, device=Q.device) if lse is True else lse
+    _check(_lib.pisa_decode_attention_noalloc(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                              _ptr(O), _ptr(L), _stream(stream)), "pisa_decode_attention_noalloc")
+    return O, L
 
 
 def check_status(ws, stream=None) -> tuple[int, int]:

@@ -1,0 +1,101 @@
+// Decode attention for callers that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc at all: code that runs inside another
+// framework's memory pool, a plugin that owns no allocator, or a serving loop
+// that must not allocate once it is running. For them,
+// pisa_decode_attention_noalloc runs the same split-KV decode kernels as
+// pisa_sparse_attention, with the split partials and the status word in a
+// fixed array that is part of this library (kNoAllocScratchBytes, 8 MiB).
+// Every GPU that loads the library holds that array until the process exits.
+//
+// Host code cannot pass the array's name to a kernel (on the host it only
+// stands in for the symbol), so the first call on each device looks up its
+// device address with cudaGetSymbolAddress, with that device current, and
+// keeps it. Every call on a device shares the one array: two calls whose
+// kernels overlap on the GPU (different streams, no ordering between them)
+// race on it.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "pisa.h"
+#include "pisa_internal.h"
+
+namespace pisa {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+constexpr int kNoAllocMaxDevices = 256;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device (looked up once per device).
+static cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace pisa
+
+using namespace pisa;
+
+extern "C" pisa_status pisa_decode_attention_noalloc(const pisa_shape* shape, const void* Q, const void* K,
+                                                     const void* V, const int32_t* idx, void* O, float* lse,
+                                                     pisa_stream_t stream) {
+    Plan pl;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (!pl.decode) return PISA_ERR_INVALID_ARG;
+    const auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    if (Q == nullptr || K == nullptr || V == nullptr || idx == nullptr || O == nullptr || misaligned(Q) ||
+        misaligned(K) || misaligned(V) || misaligned(O) || misaligned(idx))
+        return PISA_ERR_INVALID_ARG;
+    const size_t part_bytes =
+        static_cast<size_t>(pl.B) * pl.Hsel * pl.dec_splits * pl.gsel * (pl.D + 2) * sizeof(float);
+    if (kStatusBytes + part_bytes > kNoAllocScratchBytes) return PISA_ERR_WORKSPACE;
+
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return PISA_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the status word keeps the previous call's contents: it must start at zero
+    if (cudaMemsetAsync(scratch, 0, kStatusBytes, st) != cudaSuccess) return PISA_ERR_CUDA;
+
+    DecodeParams d{};
+    d.Q = static_cast<const __nv_bfloat16*>(Q);
+    d.K = static_cast<const __nv_bfloat16*>(K);
+    d.V = static_cast<const __nv_bfloat16*>(V);
+    d.idx = idx;
+    d.part = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kStatusBytes);
+    d.O = static_cast<__nv_bfloat16*>(O);
+    d.lse = lse;
+    d.status = static_cast<uint32_t*>(scratch);
+    d.Hq = pl.Hq;
+    d.Hkv = pl.Hkv;
+    d.g = pl.g;
+    d.N = pl.N;
+    d.n0 = pl.n0;
+    d.D = pl.D;
+    d.blk = pl.blk;
+    d.topk = pl.topk;
+    d.per_qhead = pl.per_qhead;
+    d.Hsel = pl.Hsel;
+    d.gh = pl.gsel;
+    d.bps = pl.dec_bps;
+    d.splits = pl.dec_splits;
+    d.scale_log2 = pl.scale * 1.4426950408889634f;
+    int32_t launches = 0;
+    return launch_attn_decode(pl, d, st, &launches) ? PISA_OK : PISA_ERR_CUDA;
+}

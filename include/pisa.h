@@ -162,6 +162,31 @@ PISA_API pisa_status pisa_forward(const pisa_shape *shape, const void *Q, const 
                          void *O, float *lse, int32_t *idx_out, void *ws, size_t ws_bytes,
                          pisa_stream_t stream);
 
+/* Decode attention that allocates nothing. The paper has no counterpart: this
+ * is a convenience for callers that may not call cudaMalloc, such as code
+ * running inside another framework's memory pool, a plugin without an
+ * allocator of its own, or a serving loop that must not allocate once running.
+ * It computes exactly what pisa_sparse_attention computes for a decode shape
+ * (seq_q == 1), with the same kernels, but keeps the split-KV partials and the
+ * status word in a fixed 8 MiB device array built into the library instead of
+ * a caller workspace. The caller still passes Q, K, V, idx, O and lse (lse may
+ * be NULL), laid out as for pisa_sparse_attention.
+ *   - Every GPU that loads the library holds the 8 MiB array until exit.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current and keeps it; make that first call before any stream
+ *     capture.
+ *   - Shapes whose partials need more than the array holds (batch x Hsel x
+ *     ceil(topk/4) x g x (head_dim+2) x 4 bytes, plus 256) return
+ *     PISA_ERR_WORKSPACE; non-decode shapes return PISA_ERR_INVALID_ARG.
+ *   - Calls share the array: calls whose kernels overlap on the GPU race on it.
+ *     The status word is cleared at the start of each call; errors the kernels
+ *     record there are not reported, and pisa_last_launch_count does not count
+ *     this call.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+PISA_API pisa_status pisa_decode_attention_noalloc(const pisa_shape *shape, const void *Q, const void *K,
+                                                   const void *V, const int32_t *idx, void *O, float *lse,
+                                                   pisa_stream_t stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace status word since the last call (PISA_OK if none) and clears it.
  * `detail`, if not NULL, receives a code locating the error (kernel and wait site). */
