@@ -20,10 +20,17 @@
 //   softmax reads S, finds the row max, keeps a running max that only moves
 //   when the new max exceeds it by more than 2^8 (the output and the row sum
 //   are rescaled then), writes P = exp2(S*c - m) as bf16 into shared memory
+//   (two P buffers per tile, so P for block j+1 can be written while P.V of
+//   block j still reads the other one)
 //   O[h] += P_h V_j                 (tcgen05, M=128, N=D, K=b, fp32 in TMEM)
 // The MMA lane issues S for block j+1 before O for block j, so the tensor
 // core works on one tile while the softmax warps work on the other. No score
 // ever leaves TMEM/shared memory; O is normalised once at the end.
+//
+// Softmax arithmetic per row and block: a three-input max tree, packed fp32
+// pair instructions (f32x2) for the scale-and-subtract and the row sum, and
+// the exponentials split between the MUFU unit (two thirds) and a polynomial
+// on the FMA pipes (one third), which balances the two.
 //
 // Shared memory operands use the 128-byte swizzle: Q, K and P are K-major
 // (head dim / key index contiguous), V is read MN-major straight from its
@@ -41,11 +48,12 @@ struct PrefillCfg {
     static constexpr int BS = BLK / 64;                // 128-byte column tiles along the key block
     static constexpr int SUB = 128 * 128;              // one [128 rows x 128 B] operand tile
     static constexpr int Q_BYTES = NM * DS * SUB;
-    static constexpr int P_BYTES = NM * BS * SUB;
+    static constexpr int P_BUF = NM * BS * SUB;         // one P buffer (all tiles)
+    static constexpr int P_BYTES = 2 * P_BUF;
     static constexpr int KV_SUB = BLK * 128;           // one [BLK rows x 128 B] tile
     static constexpr int KV_BYTES = DS * KV_SUB;       // a whole K (or V) block
-    static constexpr int MAX_LIST = 2048;              // selected blocks per query block
-    static constexpr int AUX = 512 + MAX_LIST * 4;     // barriers, TMEM slot, block list
+    static constexpr int MAX_LIST = kMaxPrefillTopk;   // selected blocks per query block
+    static constexpr int AUX = 256 + MAX_LIST * 4;     // barriers, TMEM slot, block list
     static constexpr int SMEM_LIMIT = 232448;          // 227 KB opt-in maximum
     static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - Q_BYTES - P_BYTES - AUX) / (2 * KV_BYTES);
     static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
@@ -69,6 +77,8 @@ struct PrefillCfg {
 // Lazy rescale threshold (log2 units): the running max is kept until a new
 // row max exceeds it by this much, so probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f;
+// Pairs of scores k with k % kPolyMod == kPolyMod - 1 take the FMA-pipe exp2.
+constexpr int kPolyMod = 3;
 
 template <int D, int BLK, int NM>
 __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
@@ -89,12 +99,12 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     uint64_t* kv_empty = v_full + C::NST;           // NST
     uint64_t* s_full = kv_empty + C::NST;           // NM*2
     uint64_t* s_empty = s_full + NM * 2;            // NM*2
-    uint64_t* p_full = s_empty + NM * 2;            // NM
-    uint64_t* o_done = p_full + NM;                 // NM
-    uint64_t* mma_final = o_done + NM;              // 1
+    uint64_t* p_full = s_empty + NM * 2;            // NM*2: P buffer written by the softmax
+    uint64_t* p_empty = p_full + NM * 2;            // NM*2: P.V that read the buffer completed
+    uint64_t* mma_final = p_empty + NM * 2;         // 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
     int32_t* s_nsel = reinterpret_cast<int32_t*>(tmem_slot + 1);
-    int32_t* list = reinterpret_cast<int32_t*>(aux + 512);
+    int32_t* list = reinterpret_cast<int32_t*>(aux + 256);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -119,8 +129,10 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             mbar_init(s_full + 2 * h + 1, 1);
             mbar_init(s_empty + 2 * h, 128);
             mbar_init(s_empty + 2 * h + 1, 128);
-            mbar_init(p_full + h, 128);
-            mbar_init(o_done + h, 1);
+            mbar_init(p_full + 2 * h, 128);
+            mbar_init(p_full + 2 * h + 1, 128);
+            mbar_init(p_empty + 2 * h, 1);
+            mbar_init(p_empty + 2 * h + 1, 1);
         }
         mbar_init(mma_final, 1);
         fence_barrier_init();
@@ -219,19 +231,22 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                 if (j >= 1) {
                     const int jj = j - 1, st = jj % C::NST;
                     if (!(ok = mbar_wait(v_full + st, (jj / C::NST) & 1, p.status, detail_base | 0x13u))) break;
+                    const int pb = jj & 1;
                     for (int h = 0; h < NM; ++h) {
-                        if (!(ok = mbar_wait(p_full + h, jj & 1, p.status, detail_base | 0x14u))) break;
+                        if (!(ok = mbar_wait(p_full + 2 * h + pb, (jj >> 1) & 1, p.status, detail_base | 0x14u)))
+                            break;
                         tc_fence_after();
                         const uint32_t d_tmem = tm + C::O_COL + h * D;
 #pragma unroll
                         for (int ks = 0; ks < BLK / 16; ++ks) {
                             const uint32_t koff = (ks % 4) * 32;
-                            const uint64_t a = smem_desc_sw128(p_addr + (h * C::BS + ks / 4) * C::SUB + koff, 16, 1024);
+                            const uint64_t a = smem_desc_sw128(
+                                p_addr + pb * C::P_BUF + (h * C::BS + ks / 4) * C::SUB + koff, 16, 1024);
                             const uint64_t bd = smem_desc_sw128(v_addr + st * C::KV_BYTES + ks * 16 * 128,
                                                                 C::KV_SUB, 1024);
                             mma_bf16_ss(d_tmem, a, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
                         }
-                        mma_commit(o_done + h);
+                        mma_commit(p_empty + 2 * h + pb);
                         issued_any_mma = true;
                     }
                     if (!ok) break;
@@ -250,6 +265,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         const int hh = R / BLK, t = R % BLK;
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const float cs = p.scale_log2;
+        const uint64_t cs2 = f2_pack(cs, cs);
         float m_used = -INFINITY, l_sum = 0.f;
         bool ok = true;
         for (int j = 0; j < nsel; ++j) {
@@ -257,24 +273,34 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             ok = mbar_wait(s_full + 2 * h + buf, (j >> 1) & 1, p.status, detail_base | 0x20u);
             if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[BLK];
+            float sv[BLK];
 #pragma unroll
             for (int c = 0; c < BLK / 32; ++c)
                 tmem_ld32(tm + lane_base + C::S_COL + (buf * NM + h) * BLK + c * 32,
-                          *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+                          *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(s_empty + 2 * h + buf);
 
-            const bool diag = p.causal && list[j] == i;
-            float mx = -INFINITY;
+            const bool diag = p.causal && list[j] == i;  // uniform across the CTA
+            if (diag) {
 #pragma unroll
-            for (int c = 0; c < BLK; ++c) {
-                float s = __uint_as_float(sr[c]);
-                if (diag && c > t) s = -INFINITY;
-                sr[c] = __float_as_uint(s);
-                mx = fmaxf(mx, s);
+                for (int c = 0; c < BLK; ++c) sv[c] = c > t ? -INFINITY : sv[c];
             }
+            // row max: eight independent three-input max chains
+            float mq[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mq[q] = sv[q];
+#pragma unroll
+            for (int c = 8; c + 16 <= BLK; c += 16) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mq[q] = fmax3(mq[q], sv[c + q], sv[c + 8 + q]);
+            }
+            if ((BLK - 8) % 16 != 0) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], sv[BLK - 8 + q]);
+            }
+            const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7])));
             const float mxs = mx * cs;
             bool resc = false;
             float m_new = m_used;
@@ -285,39 +311,56 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                 m_new = mxs;
             }
             const float alpha = resc ? fast_exp2(m_used - m_new) : 1.0f;
+            const uint64_t negm2 = f2_pack(-m_new, -m_new);
             uint32_t pk[BLK / 2];
-            float rs = 0.f;
+            uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int c = 0; c < BLK; c += 2) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), cs, -m_new));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), cs, -m_new));
-                rs += p0 + p1;
-                pk[c / 2] = pack_bf16x2(p0, p1);
+            for (int k = 0; k < BLK / 2; ++k) {
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
+                uint64_t e2;
+                if (!diag && (k % kPolyMod) == kPolyMod - 1) {
+                    e2 = exp2_poly_x2(x0, x1);
+                } else {
+                    e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+                }
+                sum2[k & 3] = f2_add(sum2[k & 3], e2);
+                float e0, e1;
+                f2_unpack(e2, e0, e1);
+                pk[k] = pack_bf16x2(e0, e1);
             }
-            if (j > 0) {
-                ok = mbar_wait(o_done + h, (j - 1) & 1, p.status, detail_base | 0x21u);
+            float r0, r1, r2, r3;
+            f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), r0, r1);
+            const float rs = r0 + r1;
+            (void)r2;
+            (void)r3;
+            if (j > 0 && __any_sync(0xFFFFFFFFu, resc)) {
+                // O must hold P.V of block j-1 before it is rescaled
+                const int pj = j - 1;
+                ok = mbar_wait(p_empty + 2 * h + (pj & 1), (pj >> 1) & 1, p.status, detail_base | 0x21u);
                 if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
                 tc_fence_after();
-                if (__any_sync(0xFFFFFFFFu, resc)) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        const uint32_t addr = tm + lane_base + C::O_COL + h * D + c * 32;
-                        tmem_ld32(addr, o);
-                        tmem_wait_ld();
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    const uint32_t addr = tm + lane_base + C::O_COL + h * D + c * 32;
+                    tmem_ld32(addr, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                        tmem_st32(addr, o);
-                    }
-                    tmem_wait_st();
+                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                    tmem_st32(addr, o);
                 }
+                tmem_wait_st();
             }
             l_sum = l_sum * alpha + rs;
             m_used = m_new;
+            // this P buffer was last read by P.V of block j-2
+            ok = mbar_wait(p_empty + 2 * h + buf, ((j >> 1) & 1) ^ 1, p.status, detail_base | 0x23u);
+            if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
             if (valid) {
 #pragma unroll
                 for (int ps = 0; ps < C::BS; ++ps) {
-                    const uint32_t rowaddr = smem_u32(Ps + (h * C::BS + ps) * C::SUB) + r * 128;
+                    const uint32_t rowaddr = smem_u32(Ps + buf * C::P_BUF + (h * C::BS + ps) * C::SUB) + r * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const uint32_t* q4 = pk + ps * 32 + c * 4;
@@ -327,14 +370,15 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full + h);
+            mbar_arrive(p_full + 2 * h + buf);
         }
         // ---------------------------------------------------------------- epilogue
         if (ok) {
             const int head = head0 + hh;
             const int64_t orow = (static_cast<int64_t>(b) * p.Hq + head) * p.N + static_cast<int64_t>(i) * BLK + t;
             if (nsel > 0) {
-                ok = mbar_wait(o_done + h, (nsel - 1) & 1, p.status, detail_base | 0x22u);
+                const int pj = nsel - 1;
+                ok = mbar_wait(p_empty + 2 * h + (pj & 1), (pj >> 1) & 1, p.status, detail_base | 0x22u);
                 ok = __all_sync(0xFFFFFFFFu, ok);
             }
             if (ok) {

@@ -69,6 +69,7 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->nqb = p->decode ? 1 : p->Nq / p->blk;
     if (p->Hsel > 65535 / 16) return PISA_ERR_UNSUPPORTED;
     if (p->decode && p->gsel > 8) return PISA_ERR_UNSUPPORTED;
+    if (!p->decode && p->topk > kMaxPrefillTopk) return PISA_ERR_UNSUPPORTED;
 
     p->dec_bps = 4;
     p->dec_splits = p->decode ? (p->topk + p->dec_bps - 1) / p->dec_bps : 0;

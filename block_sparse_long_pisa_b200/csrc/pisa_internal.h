@@ -12,6 +12,9 @@ namespace pisa {
 // Upper bound on any single pipeline wait inside a kernel (ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Selected blocks per query block the prefill attention kernel holds on chip.
+constexpr int kMaxPrefillTopk = 256;
+
 // Bytes reserved for the status word at the start of the workspace.
 constexpr size_t kStatusBytes = 256;
 

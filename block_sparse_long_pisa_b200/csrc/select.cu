@@ -12,7 +12,8 @@
 //    children are exactly the eligible nodes of this level, and skipping the
 //    coarser scores changes nothing.
 // 4. At each level every candidate gets an fp32 dot product with the query
-//    summary (one thread per candidate, float4 loads). Candidates are ranked by
+//    summary (eight lanes per candidate, so each warp load covers four whole
+//    128-byte lines of node vectors; a three-step shuffle adds the lanes). Candidates are ranked by
 //    a 64-bit key (order-preserving score bits, then inverted node index), so
 //    that a bitonic sort in shared memory orders by higher score and, on equal
 //    scores, lower index. The kept nodes' eligible children become the next
@@ -91,21 +92,6 @@ __device__ __forceinline__ int next_pow2(int n) {
 }
 
 template <int D>
-__device__ __forceinline__ float dot_row(const float* __restrict__ qs, const float* v) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < D; d += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(v + d);
-        const float4 q = *reinterpret_cast<const float4*>(qs + d);
-        a0 = fmaf(q.x, x.x, a0);
-        a1 = fmaf(q.y, x.y, a1);
-        a2 = fmaf(q.z, x.z, a2);
-        a3 = fmaf(q.w, x.w, a3);
-    }
-    return (a0 + a1) + (a2 + a3);
-}
-
-template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams p, int cap) {
     extern __shared__ __align__(16) uint8_t sm[];
     uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                         // [cap]
@@ -136,6 +122,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     }
     if (tid == 0) s_margin = __int_as_float(0x7F800000);  // +inf
     __syncthreads();
+    // this lane's slice of the query summary: dims 32k + 4*sub .. +3
+    const int sub = tid & 7;
+    float4 qv[D / 32];
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) qv[k] = *reinterpret_cast<const float4*>(qs + 32 * k + 4 * sub);
 
     // coarsest level whose eligible nodes exceed its budget
     int l0 = -1;
@@ -162,15 +153,28 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             const int n = next_pow2(ncand);
             const int64_t c_part = last / p.width[l];
             const bool has_part = min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
-            for (int t = tid; t < n; t += kSelThreads) {
-                uint64_t key = 0;
-                if (t < ncand && cand[t] >= 0) {
-                    const int32_t c = cand[t];
+            // 8 lanes per candidate: each warp load instruction covers four whole 128-byte lines
+            for (int t0 = 0; t0 < n; t0 += kSelThreads / 8) {
+                const int t = t0 + (tid >> 3);
+                const bool live = t < ncand && cand[t] >= 0;
+                const int32_t c = live ? cand[t] : 0;
+                float acc = 0.f;
+                if (live) {
                     const float* v = (has_part && c == c_part) ? part + l * D
                                                                : plane + static_cast<int64_t>(p.loff[l] + c) * D;
-                    key = rank_key(dot_row<D>(qs, v), c);
+#pragma unroll
+                    for (int k = 0; k < D / 32; ++k) {
+                        const float4 x = *reinterpret_cast<const float4*>(v + 32 * k + 4 * sub);
+                        acc = fmaf(qv[k].x, x.x, acc);
+                        acc = fmaf(qv[k].y, x.y, acc);
+                        acc = fmaf(qv[k].z, x.z, acc);
+                        acc = fmaf(qv[k].w, x.w, acc);
+                    }
                 }
-                keys[t] = key;
+                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
+                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+                if (sub == 0 && t < n) keys[t] = live ? rank_key(acc, c) : 0ull;
             }
             __syncthreads();
             const int nvalid = s_nvalid;

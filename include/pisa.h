@@ -56,7 +56,8 @@ typedef struct CUstream_st *pisa_stream_t;
  *   head_dim                 : 64 or 128.
  *   block                    : key-block size b (and query-block size for prefill): 64 or 128.
  *   factor                   : pooling factor f >= 2 between pyramid levels.
- *   topk                     : K, key blocks kept per query block, 1 <= K.
+ *   topk                     : K, key blocks kept per query block, 1 <= K; factor * K <= 4096,
+ *                              and K <= 256 for prefill (seq_q == seq_kv).
  *   causal                   : 0/1. Prefill only: query block i may use key blocks j <= i
  *                              and, inside block i, keys at or before the query.
  *   select_per_qhead         : 0 = one selection per (batch, KV head, query block) from the
