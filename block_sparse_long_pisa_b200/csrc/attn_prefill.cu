@@ -8,35 +8,43 @@
 // once by TMA and used by all rows, so GQA groups reuse each gathered byte gh
 // times.
 //
+// The selected blocks are taken in key groups of 128 keys (two 64-key blocks,
+// or one 128-key block). A tcgen05 MMA with M = 128 costs the same for N = 64
+// as for N = 128, so grouping doubles the useful work of every Q.K^T
+// instruction; P.V gets K = 128 per group.
+//
 // Warp roles (warp-specialised pipeline, all hand-off through mbarriers):
-//   warps 0 .. 4*NM-1  softmax: warp w owns TMEM lanes 32*(w%4).. of tile w/4,
-//                      one query row per thread
-//   warp 4*NM          producer: one lane issues the TMA loads (Q once, then
-//                      K and V of every selected block into an NST-deep ring)
-//   warp 4*NM+1        MMA: allocates TMEM and one lane issues tcgen05.mma
+//   warps 0 .. 8*NM-1  softmax: two warps per query row. Warp w reads TMEM
+//                      lanes 32*(w%4).. of tile (w/4)%NM and owns the 64
+//                      score columns of its half (w/(4*NM)); the partner warp
+//                      of the other half shares the rows. They exchange row
+//                      maxima and sums through shared memory and a 64-thread
+//                      named barrier, and each writes half of O at the end.
+//   warp 8*NM          producer: lane 0 streams K groups, lane 1 V groups, by
+//                      2-D TMA into NST-deep rings (each with its own empty
+//                      barrier, so K can run ahead of V)
+//   warp 8*NM+1        MMA: allocates TMEM and one lane issues tcgen05.mma
 //
-// Per selected block j and tile h:
-//   S[h][j&1] = Q_h K_j^T           (tcgen05, M=128, N=b, K=D, fp32 in TMEM)
-//   softmax reads S, finds the row max, keeps a running max that only moves
-//   when the new max exceeds it by more than 2^8 (the output and the row sum
-//   are rescaled then), writes P = exp2(S*c - m) as bf16 into shared memory
-//   (two P buffers per tile, so P for block j+1 can be written while P.V of
-//   block j still reads the other one)
-//   O[h] += P_h V_j                 (tcgen05, M=128, N=D, K=b, fp32 in TMEM)
-// The MMA lane issues S for block j+1 before O for block j, so the tensor
-// core works on one tile while the softmax warps work on the other. No score
-// ever leaves TMEM/shared memory; O is normalised once at the end.
+// Per key group g and tile h:
+//   S[h] = Q_h K_g^T     tcgen05 (A = Q and B = K from shared memory), fp32 in TMEM
+//   softmax: P = exp2(S*c - m) against the running row max m, written as bf16
+//            back into the TMEM columns of S already read (keys 0-63 into
+//            columns 0-31, keys 64-127 into columns 64-95). m moves only when a
+//            score exceeds it by more than 2^8; then that group is redone from
+//            the intact S with the new max and O and the row sums are rescaled
+//   O[h] += P_h V_g      tcgen05 with A = P read from TMEM, B = V (MN-major)
+// Because P overwrites S, a tile's next Q.K^T waits for its P.V. With two
+// tiles the MMA lane issues Q.K^T(0, g), P.V(1, g-1), Q.K^T(1, g), P.V(0, g):
+// each tile's softmax overlaps two MMAs of the other tile. No score ever
+// leaves TMEM.
 //
-// Softmax arithmetic per row and block: a three-input max tree, packed fp32
-// pair instructions (f32x2) for the scale-and-subtract and the row sum, and
-// the exponentials split between the MUFU unit (two thirds) and a polynomial
-// on the FMA pipes (one third), which balances the two.
-//
-// Shared memory operands use the 128-byte swizzle: Q, K and P are K-major
-// (head dim / key index contiguous), V is read MN-major straight from its
-// [key, dim] layout.
+// Softmax arithmetic: packed fp32 pair instructions (f32x2) for the
+// scale-and-subtract and the row sum, and the exponentials split between the
+// MUFU unit and a polynomial on the FMA pipes.
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "pisa_device.cuh"
 
@@ -45,33 +53,28 @@ namespace pisa {
 template <int D, int BLK, int NM>
 struct PrefillCfg {
     static constexpr int DS = D / 64;                  // 128-byte column tiles along the head dim
-    static constexpr int BS = BLK / 64;                // 128-byte column tiles along the key block
+    static constexpr int GB = 128 / BLK;               // selected blocks per 128-key group
     static constexpr int SUB = 128 * 128;              // one [128 rows x 128 B] operand tile
     static constexpr int Q_BYTES = NM * DS * SUB;
-    static constexpr int P_BUF = NM * BS * SUB;         // one P buffer (all tiles)
-    static constexpr int P_BYTES = 2 * P_BUF;
-    static constexpr int KV_SUB = BLK * 128;           // one [BLK rows x 128 B] tile
-    static constexpr int KV_BYTES = DS * KV_SUB;       // a whole K (or V) block
+    static constexpr int KG_BYTES = DS * SUB;          // a 128-key K (or V) group
     static constexpr int MAX_LIST = kMaxPrefillTopk;   // selected blocks per query block
-    static constexpr int AUX = 256 + MAX_LIST * 4;     // barriers, TMEM slot, block list
+    static constexpr int XCH = 2 * 2 * NM * 128 * 4;       // [parity][half][tile][row] row statistics
+    static constexpr int AUX = 512 + MAX_LIST * 4 + XCH;   // barriers, TMEM slot, block list, exchange
     static constexpr int SMEM_LIMIT = 232448;          // 227 KB opt-in maximum
-    static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - Q_BYTES - P_BYTES - AUX) / (2 * KV_BYTES);
+    static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - Q_BYTES - AUX) / (2 * KG_BYTES);
     static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-    static constexpr int SMEM = 1024 + Q_BYTES + P_BYTES + NST * 2 * KV_BYTES + AUX;
+    static constexpr int SMEM = 1024 + Q_BYTES + NST * 2 * KG_BYTES + AUX;
     static constexpr int O_COL = 0;
-    static constexpr int S_COL = NM * D;
-    static constexpr int TMEM_NEED = NM * D + 2 * NM * BLK;
-    static constexpr int TMEM_COLS = TMEM_NEED <= 32    ? 32
-                                     : TMEM_NEED <= 64  ? 64
-                                     : TMEM_NEED <= 128 ? 128
-                                     : TMEM_NEED <= 256 ? 256
-                                                        : 512;
-    static constexpr int SOFTMAX_WARPS = 4 * NM;
+    static constexpr int S_COL = NM * D;               // S/P of tile h at S_COL + 128 h
+    static constexpr int TMEM_NEED = NM * D + NM * 128;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
+    static constexpr int SOFTMAX_WARPS = 8 * NM;          // two warps per query row
     static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
     static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
     static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
-    static_assert(NST >= 2, "shared memory too small for a double-buffered K/V ring");
+    static_assert(NST >= 2, "shared memory too small for double-buffered K/V rings");
     static_assert(TMEM_NEED <= 512, "TMEM budget exceeded");
+    static_assert(BLK == 64 || BLK == 128, "key block of 64 or 128");
 };
 
 // Lazy rescale threshold (log2 units): the running max is kept until a new
@@ -88,23 +91,24 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* Qs = base;
-    uint8_t* Ps = Qs + C::Q_BYTES;
-    uint8_t* Ks = Ps + C::P_BYTES;
-    uint8_t* Vs = Ks + C::NST * C::KV_BYTES;
-    uint8_t* aux = Vs + C::NST * C::KV_BYTES;
+    uint8_t* Ks = Qs + C::Q_BYTES;
+    uint8_t* Vs = Ks + C::NST * C::KG_BYTES;
+    uint8_t* aux = Vs + C::NST * C::KG_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
-    uint64_t* q_full = bars;                        // 1
-    uint64_t* k_full = q_full + 1;                  // NST
-    uint64_t* v_full = k_full + C::NST;             // NST
-    uint64_t* kv_empty = v_full + C::NST;           // NST
-    uint64_t* s_full = kv_empty + C::NST;           // NM*2
-    uint64_t* s_empty = s_full + NM * 2;            // NM*2
-    uint64_t* p_full = s_empty + NM * 2;            // NM*2: P buffer written by the softmax
-    uint64_t* p_empty = p_full + NM * 2;            // NM*2: P.V that read the buffer completed
-    uint64_t* mma_final = p_empty + NM * 2;         // 1
+    uint64_t* q_full = bars;                  // 1
+    uint64_t* k_full = q_full + 1;            // NST
+    uint64_t* v_full = k_full + C::NST;       // NST
+    uint64_t* k_empty = v_full + C::NST;      // NST  (Q.K^T of the group completed)
+    uint64_t* v_empty = k_empty + C::NST;     // NST  (P.V of the group completed)
+    uint64_t* s_full = v_empty + C::NST;      // NM   (S of tile h in TMEM)
+    uint64_t* p_full = s_full + NM;           // NM   (P of tile h in TMEM, O rescaled)
+    uint64_t* pv_done = p_full + NM;          // NM   (P.V of tile h completed)
+    uint64_t* x_bar = pv_done + NM;           // 4*NM (two softmax warps of a row quadrant meet)
+    uint64_t* mma_final = x_bar + 4 * NM;     // 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
     int32_t* s_nsel = reinterpret_cast<int32_t*>(tmem_slot + 1);
-    int32_t* list = reinterpret_cast<int32_t*>(aux + 256);
+    int32_t* list = reinterpret_cast<int32_t*>(aux + 512);
+    float* xch = reinterpret_cast<float*>(aux + 512 + C::MAX_LIST * 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -122,18 +126,15 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(v_full + s, 1);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(v_empty + s, 1);
         }
         for (int h = 0; h < NM; ++h) {
-            mbar_init(s_full + 2 * h, 1);
-            mbar_init(s_full + 2 * h + 1, 1);
-            mbar_init(s_empty + 2 * h, 128);
-            mbar_init(s_empty + 2 * h + 1, 128);
-            mbar_init(p_full + 2 * h, 128);
-            mbar_init(p_full + 2 * h + 1, 128);
-            mbar_init(p_empty + 2 * h, 1);
-            mbar_init(p_empty + 2 * h + 1, 1);
+            mbar_init(s_full + h, 1);
+            mbar_init(p_full + h, 256);
+            mbar_init(pv_done + h, 1);
         }
+        for (int q = 0; q < 4 * NM; ++q) mbar_init(x_bar + q, 64);
         mbar_init(mma_final, 1);
         fence_barrier_init();
     }
@@ -148,7 +149,8 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             const bool ok = j >= 0 && j < p.n0 && (!p.causal || j <= i);
             if (t < p.topk && j >= 0 && !ok) record_error(p.status, PISA_ERR_BAD_INDEX, detail_base | 0xB0u);
             const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
-            if (ok && cnt + __popc(m & ((1u << lane) - 1u)) < C::MAX_LIST) list[cnt + __popc(m & ((1u << lane) - 1u))] = j;
+            const int pos = cnt + __popc(m & ((1u << lane) - 1u));
+            if (ok && pos < C::MAX_LIST) list[pos] = j;
             cnt += __popc(m);
         }
         if (lane == 0) *s_nsel = cnt < C::MAX_LIST ? cnt : C::MAX_LIST;
@@ -158,238 +160,303 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
     const int nsel = *s_nsel;
+    const int ngroups = (nsel + C::GB - 1) / C::GB;
 
-    int issued_last[C::NST];  // producer: last ring use issued per stage (-1 = none)
-#pragma unroll
-    for (int s = 0; s < C::NST; ++s) issued_last[s] = -1;
+    int issued_last = -1;  // producer lanes: last group whose copies they started
     bool issued_any_mma = false;
 
     if (warp == C::PRODUCER_WARP) {
-        if (lane == 0 && nsel > 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.gh * BLK * D * 2));
-            for (int hh = 0; hh < p.gh; ++hh) {
-                const int r0 = hh * BLK;
-                const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
-                                                  static_cast<int64_t>(i) * BLK);
+        if (lane < 2 && ngroups > 0) {
+            const bool is_k = lane == 0;
+            const void* tmap = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+            uint8_t* ring = is_k ? Ks : Vs;
+            uint64_t* full = is_k ? k_full : v_full;
+            uint64_t* empty = is_k ? k_empty : v_empty;
+            prefetch_tmap(tmap);
+            if (is_k) {
+                prefetch_tmap(&tmQ);
+                mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.gh * BLK * D * 2));
+                for (int hh = 0; hh < p.gh; ++hh) {
+                    const int r0 = hh * BLK;
+                    const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
+                                                      static_cast<int64_t>(i) * BLK);
 #pragma unroll
-                for (int s = 0; s < C::DS; ++s)
-                    tma_load_2d(Qs + ((r0 / 128) * C::DS + s) * C::SUB + (r0 % 128) * 128, &tmQ, s * 64, qrow,
-                                q_full);
+                    for (int s = 0; s < C::DS; ++s)
+                        tma_load_2d(Qs + ((r0 / 128) * C::DS + s) * C::SUB + (r0 % 128) * 128, &tmQ, s * 64, qrow,
+                                    q_full);
+                }
             }
-            for (int j = 0; j < nsel; ++j) {
-                const int st = j % C::NST, use = j / C::NST;
-                if (!mbar_wait(kv_empty + st, (use & 1) ^ 1, p.status, detail_base | 0x01u)) break;
-                const int krow = static_cast<int>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N +
-                                                  static_cast<int64_t>(list[j]) * BLK);
-                mbar_arrive_expect_tx(k_full + st, C::KV_BYTES);
+            for (int g = 0; g < ngroups; ++g) {
+                const int st = g % C::NST, use = g / C::NST;
+                if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
+                const int nb = min(C::GB, nsel - g * C::GB);
+                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * BLK * D * 2));
+                for (int u = 0; u < nb; ++u) {
+                    const int krow = static_cast<int>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N +
+                                                      static_cast<int64_t>(list[g * C::GB + u]) * BLK);
 #pragma unroll
-                for (int s = 0; s < C::DS; ++s)
-                    tma_load_2d(Ks + st * C::KV_BYTES + s * C::KV_SUB, &tmK, s * 64, krow, k_full + st);
-                mbar_arrive_expect_tx(v_full + st, C::KV_BYTES);
-#pragma unroll
-                for (int s = 0; s < C::DS; ++s)
-                    tma_load_2d(Vs + st * C::KV_BYTES + s * C::KV_SUB, &tmV, s * 64, krow, v_full + st);
-                issued_last[st] = use;
+                    for (int s = 0; s < C::DS; ++s)
+                        tma_load_2d(ring + st * C::KG_BYTES + s * C::SUB + u * BLK * 128, tmap, s * 64, krow,
+                                    full + st);
+                }
+                issued_last = g;
             }
         }
         __syncwarp();
     } else if (warp == C::MMA_WARP) {
-        if (lane == 0 && nsel > 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BLK, 0, 0);
+        if (lane == 0 && ngroups > 0) {
+            const uint32_t q_addr = smem_u32(Qs), k_addr = smem_u32(Ks), v_addr = smem_u32(Vs);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t q_addr = smem_u32(Qs), k_addr = smem_u32(Ks), v_addr = smem_u32(Vs),
-                           p_addr = smem_u32(Ps);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
             tc_fence_after();
-            for (int j = 0; ok && j <= nsel; ++j) {
-                if (j < nsel) {
-                    const int st = j % C::NST;
-                    if (!(ok = mbar_wait(k_full + st, (j / C::NST) & 1, p.status, detail_base | 0x11u))) break;
-                    const int buf = j & 1;
-                    for (int h = 0; h < NM; ++h) {
-                        if (!(ok = mbar_wait(s_empty + 2 * h + buf, ((j >> 1) & 1) ^ 1, p.status,
-                                             detail_base | 0x12u)))
-                            break;
-                        tc_fence_after();
-                        const uint32_t d_tmem = tm + C::S_COL + (buf * NM + h) * BLK;
+            // S[h] = Q_h K_g^T (after P.V of group g-1 on tile h has released the TMEM columns)
+            auto qk = [&](int g, int h) -> bool {
+                const int st = g % C::NST;
+                if (g > 0 && !mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x12u)) return false;
+                tc_fence_after();
+                const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
+                const uint32_t idesc_qk = idesc_bf16_f32(128, ncols, 0, 0);
+                const uint32_t d_tmem = tm + C::S_COL + h * 128;
 #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t koff = (ks % 4) * 32;
-                            const uint64_t a = smem_desc_sw128(q_addr + (h * C::DS + ks / 4) * C::SUB + koff, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(
-                                k_addr + st * C::KV_BYTES + (ks / 4) * C::KV_SUB + koff, 16, 1024);
-                            mma_bf16_ss(d_tmem, a, bd, idesc_qk, ks > 0 ? 1u : 0u);
-                        }
-                        mma_commit(s_full + 2 * h + buf);
-                        issued_any_mma = true;
-                    }
-                    if (!ok) break;
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t koff = (ks % 4) * 32;
+                    const uint64_t a = smem_desc_sw128(q_addr + (h * C::DS + ks / 4) * C::SUB + koff, 16, 1024);
+                    const uint64_t bd =
+                        smem_desc_sw128(k_addr + st * C::KG_BYTES + (ks / 4) * C::SUB + koff, 16, 1024);
+                    mma_bf16_ss(d_tmem, a, bd, idesc_qk, ks > 0 ? 1u : 0u);
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, st = jj % C::NST;
-                    if (!(ok = mbar_wait(v_full + st, (jj / C::NST) & 1, p.status, detail_base | 0x13u))) break;
-                    const int pb = jj & 1;
-                    for (int h = 0; h < NM; ++h) {
-                        if (!(ok = mbar_wait(p_full + 2 * h + pb, (jj >> 1) & 1, p.status, detail_base | 0x14u)))
-                            break;
-                        tc_fence_after();
-                        const uint32_t d_tmem = tm + C::O_COL + h * D;
-#pragma unroll
-                        for (int ks = 0; ks < BLK / 16; ++ks) {
-                            const uint32_t koff = (ks % 4) * 32;
-                            const uint64_t a = smem_desc_sw128(
-                                p_addr + pb * C::P_BUF + (h * C::BS + ks / 4) * C::SUB + koff, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(v_addr + st * C::KV_BYTES + ks * 16 * 128,
-                                                                C::KV_SUB, 1024);
-                            mma_bf16_ss(d_tmem, a, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        mma_commit(p_empty + 2 * h + pb);
-                        issued_any_mma = true;
-                    }
-                    if (!ok) break;
-                    mma_commit(kv_empty + st);
+                mma_commit(s_full + h);
+                issued_any_mma = true;
+                return true;
+            };
+            // O[h] += P_h V_g (P in TMEM: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
+            auto pv = [&](int g, int h) -> bool {
+                const int st = g % C::NST;
+                if (!mbar_wait(p_full + h, g & 1, p.status, detail_base | 0x14u)) return false;
+                tc_fence_after();
+                const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
+                const uint32_t d_tmem = tm + C::O_COL + h * D;
+                const uint32_t a_tmem = tm + C::S_COL + h * 128;
+                for (int ks = 0; ks < ncols / 16; ++ks) {
+                    const uint64_t bd = smem_desc_sw128(v_addr + st * C::KG_BYTES + ks * 16 * 128, C::SUB, 1024);
+                    const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
+                    mma_bf16_ts(d_tmem, a_tmem + acol, bd, idesc_pv, (g > 0 || ks > 0) ? 1u : 0u);
                 }
+                mma_commit(pv_done + h);
+                return true;
+            };
+            for (int g = 0; ok && g < ngroups; ++g) {
+                const int st = g % C::NST, ph = (g / C::NST) & 1;
+                if (!(ok = mbar_wait(k_full + st, ph, p.status, detail_base | 0x11u))) break;
+                if (!(ok = qk(g, 0))) break;
+                if (NM == 2) {
+                    if (g > 0) {
+                        // P.V(1, g-1) goes between the two Q.K^T of group g
+                        if (!(ok = pv(g - 1, 1))) break;
+                        mma_commit(v_empty + (g - 1) % C::NST);
+                    }
+                    if (!(ok = qk(g, 1))) break;
+                }
+                mma_commit(k_empty + st);
+                if (!(ok = mbar_wait(v_full + st, ph, p.status, detail_base | 0x13u))) break;
+                if (!(ok = pv(g, 0))) break;
+                if (NM == 1) mma_commit(v_empty + st);
+            }
+            if (ok && NM == 2) {
+                if (pv(ngroups - 1, 1)) mma_commit(v_empty + (ngroups - 1) % C::NST);
             }
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax warps
-        const int h = warp / 4;
+        const int h = (warp / 4) % NM;
         const int qd = warp % 4;
+        const int ch = warp / (4 * NM);   // column half: keys [64 ch, 64 ch + 64) of every group
         const int r = qd * 32 + lane;     // row inside tile h
         const int R = h * 128 + r;        // row inside the CTA
         const bool valid = R < p.gh * BLK;
         const int hh = R / BLK, t = R % BLK;
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+        const uint32_t s_tmem = tm + lane_base + C::S_COL + h * 128 + ch * 64;
+        // Row statistics meet through shared memory: this warp writes its value, both warps
+        // of the row quadrant arrive on x_bar, and each reads the other's value. The slots
+        // alternate with the exchange count, so a slot is rewritten only after the partner
+        // has passed the next exchange (and so has read it).
+        uint64_t* xb = x_bar + h * 4 + qd;
+        uint32_t n_xch = 0;
+        auto exchange = [&](float mine_v, float& other) -> bool {
+            float* slot = xch + (((n_xch & 1) * 2 + ch) * NM + h) * 128 + r;
+            *slot = mine_v;
+            mbar_arrive(xb);
+            const bool w = mbar_wait(xb, n_xch & 1, p.status, detail_base | 0x24u);
+            other = *(xch + (((n_xch & 1) * 2 + (ch ^ 1)) * NM + h) * 128 + r);
+            ++n_xch;
+            return w;
+        };
         const float cs = p.scale_log2;
         const uint64_t cs2 = f2_pack(cs, cs);
-        float m_used = -INFINITY, l_sum = 0.f;
+        float m_used = -INFINITY, l_part = 0.f;
         bool ok = true;
-        for (int j = 0; j < nsel; ++j) {
-            const int buf = j & 1;
-            ok = mbar_wait(s_full + 2 * h + buf, (j >> 1) & 1, p.status, detail_base | 0x20u);
+        for (int g = 0; g < ngroups; ++g) {
+            const int nb = min(C::GB, nsel - g * C::GB);
+            const int ncols = nb * BLK;
+            const int mine = max(0, min(64, ncols - ch * 64));  // columns of this half that hold keys
+            ok = mbar_wait(s_full + h, g & 1, p.status, detail_base | 0x20u);
             if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
             tc_fence_after();
-            float sv[BLK];
-#pragma unroll
-            for (int c = 0; c < BLK / 32; ++c)
-                tmem_ld32(tm + lane_base + C::S_COL + (buf * NM + h) * BLK + c * 32,
-                          *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(s_empty + 2 * h + buf);
-
-            const bool diag = p.causal && list[j] == i;  // uniform across the CTA
-            if (diag) {
-#pragma unroll
-                for (int c = 0; c < BLK; ++c) sv[c] = c > t ? -INFINITY : sv[c];
+            int diag_lo = 128;  // first column of the diagonal block, 128 if none
+            if (p.causal) {
+                for (int u = 0; u < nb; ++u)
+                    if (list[g * C::GB + u] == i) diag_lo = u * BLK;
             }
-            // row max: eight independent three-input max chains
-            float mq[8];
+            const bool any_mask = ncols < 128 || diag_lo < 128;  // uniform across the CTA
+            uint32_t pk[32];                                     // this half's P, bf16 pairs
+            uint64_t sum2[2] = {0ull, 0ull};
+            // exp2 of one 32-column chunk against the reference max; returns the chunk's max x.
+            // TRACK and MASKED are compile-time, so the unrolled pair loop has no branches and
+            // the compiler can interleave the sixteen independent pair chains.
+            auto chunk_exp = [&](int c, float m_ref, auto track_c, auto masked_c) -> float {
+                constexpr bool TRACK = decltype(track_c)::value;
+                constexpr bool MASKED = decltype(masked_c)::value;
+                float sv[32];
+                tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                tmem_wait_ld();
+                if (MASKED) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) mq[q] = sv[q];
-#pragma unroll
-            for (int c = 8; c + 16 <= BLK; c += 16) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) mq[q] = fmax3(mq[q], sv[c + q], sv[c + 8 + q]);
-            }
-            if ((BLK - 8) % 16 != 0) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], sv[BLK - 8 + q]);
-            }
-            const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7])));
-            const float mxs = mx * cs;
-            bool resc = false;
-            float m_new = m_used;
-            if (j == 0) {
-                m_new = mxs;
-            } else if (mxs > m_used + kRescaleThreshold) {
-                resc = true;
-                m_new = mxs;
-            }
-            const float alpha = resc ? fast_exp2(m_used - m_new) : 1.0f;
-            const uint64_t negm2 = f2_pack(-m_new, -m_new);
-            uint32_t pk[BLK / 2];
-            uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-            for (int k = 0; k < BLK / 2; ++k) {
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
-                uint64_t e2;
-                if (!diag && (k % kPolyMod) == kPolyMod - 1) {
-                    e2 = exp2_poly_x2(x0, x1);
-                } else {
-                    e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
-                }
-                sum2[k & 3] = f2_add(sum2[k & 3], e2);
-                float e0, e1;
-                f2_unpack(e2, e0, e1);
-                pk[k] = pack_bf16x2(e0, e1);
-            }
-            float r0, r1, r2, r3;
-            f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), r0, r1);
-            const float rs = r0 + r1;
-            (void)r2;
-            (void)r3;
-            if (j > 0 && __any_sync(0xFFFFFFFFu, resc)) {
-                // O must hold P.V of block j-1 before it is rescaled
-                const int pj = j - 1;
-                ok = mbar_wait(p_empty + 2 * h + (pj & 1), (pj >> 1) & 1, p.status, detail_base | 0x21u);
-                if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    const uint32_t addr = tm + lane_base + C::O_COL + h * D + c * 32;
-                    tmem_ld32(addr, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                    tmem_st32(addr, o);
-                }
-                tmem_wait_st();
-            }
-            l_sum = l_sum * alpha + rs;
-            m_used = m_new;
-            // this P buffer was last read by P.V of block j-2
-            ok = mbar_wait(p_empty + 2 * h + buf, ((j >> 1) & 1) ^ 1, p.status, detail_base | 0x23u);
-            if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-            if (valid) {
-#pragma unroll
-                for (int ps = 0; ps < C::BS; ++ps) {
-                    const uint32_t rowaddr = smem_u32(Ps + buf * C::P_BUF + (h * C::BS + ps) * C::SUB) + r * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t* q4 = pk + ps * 32 + c * 4;
-                        st_shared_v4(rowaddr + ((c ^ (r & 7)) << 4), q4[0], q4[1], q4[2], q4[3]);
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = ch * 64 + c * 32 + k;
+                        if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
                     }
                 }
+                const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+                float xm = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int kk = c * 16 + k;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
+                    if (TRACK) xm = fmax3(xm, x0, x1);
+                    uint64_t e2;
+                    if (!MASKED && (kk % kPolyMod) == kPolyMod - 1) {
+                        e2 = exp2_poly_x2(x0, x1);
+                    } else {
+                        e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+                    }
+                    sum2[k & 1] = f2_add(sum2[k & 1], e2);
+                    float e0, e1;
+                    f2_unpack(e2, e0, e1);
+                    pk[kk] = pack_bf16x2(e0, e1);
+                }
+                return xm;
+            };
+            // fast path: probabilities against the running max, valid while no score of the
+            // row (in either half) exceeds it by more than the rescale threshold
+            bool redo = g == 0;
+            if (!redo) {
+                float xmax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    if (c * 32 < mine)
+                        xmax = fmaxf(xmax, any_mask ? chunk_exp(c, m_used, std::true_type{}, std::true_type{})
+                                                    : chunk_exp(c, m_used, std::true_type{}, std::false_type{}));
+                float other;
+                ok = exchange(xmax, other);
+                if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+                xmax = fmaxf(xmax, other);
+                redo = __any_sync(0xFFFFFFFFu, xmax > kRescaleThreshold);
             }
-            fence_proxy_async_smem();
+            float alpha = 1.0f, m_new = m_used;
+            if (redo) {
+                // slow path (first group, or the max grew): the true row max, then the exponentials again
+                float mq[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mq[q] = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (c * 32 < mine) {
+                        float sv[32];
+                        tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                        tmem_wait_ld();
+                        if (any_mask) {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) {
+                                const int col = ch * 64 + c * 32 + k;
+                                if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            mq[q] = fmax3(mq[q], sv[q], fmaxf(sv[8 + q], fmaxf(sv[16 + q], sv[24 + q])));
+                    }
+                }
+                float mxs = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7]))) * cs;
+                float other;
+                ok = exchange(mxs, other);
+                if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+                mxs = fmaxf(mxs, other);
+                const bool resc = g > 0 && mxs > m_used + kRescaleThreshold;
+                m_new = (g == 0 || resc) ? mxs : m_used;
+                alpha = resc ? fast_exp2(m_used - m_new) : 1.0f;
+                if (g > 0 && __any_sync(0xFFFFFFFFu, resc)) {
+                    // O holds P.V of every earlier group (its completion preceded this S); this warp
+                    // rescales its half of the columns
+                    ok = mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x21u);
+                    if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[16];
+                        const uint32_t addr = tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 16;
+                        tmem_ld16(addr, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st16(addr, o);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 2; ++k) sum2[k] = 0ull;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    if (c * 32 < mine) {
+                        if (any_mask)
+                            chunk_exp(c, m_new, std::false_type{}, std::true_type{});
+                        else
+                            chunk_exp(c, m_new, std::false_type{}, std::false_type{});
+                    }
+            }
+            // P overwrites this half's S columns, already read: 64 scores -> 32 columns
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                if (c * 32 < mine) tmem_st16(s_tmem + c * 16, *reinterpret_cast<uint32_t(*)[16]>(pk + c * 16));
+            float r0, r1;
+            f2_unpack(f2_add(sum2[0], sum2[1]), r0, r1);
+            l_part = l_part * alpha + (r0 + r1);
+            m_used = m_new;
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full + 2 * h + buf);
+            mbar_arrive(p_full + h);
         }
         // ---------------------------------------------------------------- epilogue
         if (ok) {
             const int head = head0 + hh;
             const int64_t orow = (static_cast<int64_t>(b) * p.Hq + head) * p.N + static_cast<int64_t>(i) * BLK + t;
-            if (nsel > 0) {
-                const int pj = nsel - 1;
-                ok = mbar_wait(p_empty + 2 * h + (pj & 1), (pj >> 1) & 1, p.status, detail_base | 0x22u);
+            if (ngroups > 0) {
+                ok = mbar_wait(pv_done + h, (ngroups - 1) & 1, p.status, detail_base | 0x22u);
                 ok = __all_sync(0xFFFFFFFFu, ok);
             }
+            float l_other = 0.f;
+            if (ok) ok = __all_sync(0xFFFFFFFFu, exchange(l_part, l_other));
+            const float l_sum = l_part + l_other;
             if (ok) {
                 tc_fence_after();
-                const float inv = nsel > 0 ? 1.0f / l_sum : 0.f;
-                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+                const float inv = ngroups > 0 ? 1.0f / l_sum : 0.f;
+                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D + ch * (D / 2));
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t o[32];
-                    if (nsel > 0) {
-                        tmem_ld32(tm + lane_base + C::O_COL + h * D + c * 32, o);
+                    if (ngroups > 0) {
+                        tmem_ld32(tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 32, o);
                         tmem_wait_ld();
                     } else {
 #pragma unroll
@@ -407,22 +474,20 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                         }
                     }
                 }
-                if (valid && p.lse != nullptr)
-                    p.lse[orow] = nsel > 0 ? (m_used + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+                if (valid && ch == 0 && p.lse != nullptr)
+                    p.lse[orow] = ngroups > 0 ? (m_used + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             }
         }
     }
 
     // ---------------------------------------------------------------- teardown
     __syncthreads();
-    if (warp == C::PRODUCER_WARP && lane == 0) {
+    if (warp == C::PRODUCER_WARP && lane < 2 && issued_last >= 0) {
         // every TMA load this CTA issued has landed before shared memory is released
-        for (int s = 0; s < C::NST; ++s) {
-            if (issued_last[s] < 0) continue;
-            mbar_wait(k_full + s, issued_last[s] & 1, p.status, detail_base | 0x30u);
-            mbar_wait(v_full + s, issued_last[s] & 1, p.status, detail_base | 0x31u);
-        }
-        if (nsel > 0) mbar_wait(q_full, 0, p.status, detail_base | 0x32u);
+        uint64_t* full = lane == 0 ? k_full : v_full;
+        for (int g = max(0, issued_last - C::NST + 1); g <= issued_last; ++g)
+            mbar_wait(full + g % C::NST, (g / C::NST) & 1, p.status, detail_base | 0x30u);
+        if (lane == 0) mbar_wait(q_full, 0, p.status, detail_base | 0x32u);
     }
     if (warp == C::MMA_WARP && lane == 0 && issued_any_mma) {
         mma_commit(mma_final);
