@@ -355,11 +355,92 @@ def run_gpu(args, world, rank, local):
 
 def bench_workload(args):
     w = workloads.WORKLOADS[args.workload]
-    if w.decode:
-        raise SystemExit("bench.py times prefill workloads; decode is covered by the parity tests")
     if args.seq:
         w = w.replace(seq_q=args.seq, seq_kv=args.seq, name=f"{w.name}@N={args.seq}")
     return w
+
+
+def run_decode(args, world, rank, local):
+    """Decode step: query summaries + pyramid descent + split-KV attention (pyramid prebuilt).
+
+    Reported separately from the prefill line. The pyramid of the KV cache is built once
+    before timing (a prefill-side cost). Roofline: HBM bytes of the selected K/V blocks
+    plus the pyramid nodes the descent scores, plus q, o and the index rows.
+    """
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = rank_workload(bench_workload(args), rank)
+    shape = pisa.Shape.of(w)
+    q, k, v = (workloads.device_tensor(w, t, dev) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, dev)
+    pyr = pisa.build_pyramid(shape, k)
+    idx = torch.empty((w.batch, shape.hsel, 1, w.topk), dtype=torch.int32, device=dev)
+    O = torch.empty_like(q)
+    lse = torch.empty((w.batch, w.heads_q, 1), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches = [0]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        pisa.select_blocks(shape, q, pyr, ws, idx=idx)
+        launches[0] += pisa.last_launch_count()
+        if ev is not None:
+            ev[1].record(stream)
+        pisa.sparse_attention(shape, q, k, v, idx, ws, O=O, lse=lse)
+        launches[0] += pisa.last_launch_count()
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches[0] = 0
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clock = ClockSampler(local)
+    if rank == 0:
+        clock.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(events[s_])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = clock.stop() if rank == 0 else None
+    pisa.raise_on_device_error(ws, "decode")
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
+    n_sel = int((idx >= 0).sum().item())
+    kv_bytes = n_sel * w.block * w.head_dim * 2 * 2
+    sizes, _ = pisa.level_layout(shape)
+    node_bytes = scored_candidates(shape, sizes) * w.head_dim * 4  # pyramid node vectors the descent reads
+    small = q.numel() * 2 * 2 + idx.numel() * 4 + lse.numel() * 4
+    pk, how = peaks()
+    total_bytes = kv_bytes + node_bytes + small
+    if rank != 0:
+        return
+    line = {
+        "metric": "decode tokens/s (one query token per sequence, KV 131072)", "value": w.batch * world / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy, bf16 RNE)",
+        "config": {"workload": f"{w.name}: {w.batch} sequences x 1 query token, KV {w.seq_kv}, Hq={w.heads_q} "
+                               f"Hkv={w.heads_kv} D={w.head_dim} block={w.block} factor={w.factor} K={w.topk}, "
+                               f"pyramid prebuilt", "global_batch": w.batch * world, "seq_len": w.seq_kv,
+                   "parallelism": f"replicas x{world}"},
+        "stages_ms": {"select": sel_ms, "attention": att_ms},
+        "roofline": {"bound": "hbm", "achieved": total_bytes / (ms_step / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": total_bytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
+                     "bytes_per_step": total_bytes, "peak_source": f"{how} HBM copy", "traffic": None},
+        "gpu_launches": launches[0], "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def scored_candidates(shape, sizes) -> int:
@@ -400,7 +481,10 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_gpu(args, world, rank, local)
+        if workloads.WORKLOADS[args.workload].decode:
+            run_decode(args, world, rank, local)
+        else:
+            run_gpu(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -1,0 +1,111 @@
+"""Full-size workloads on the GPU, checked against the oracle on sampled outputs.
+
+Each workload runs at its full size in the launch configuration bench.py
+times (pisa_build_pyramid, pisa_select_blocks, pisa_sparse_attention on one
+stream; pisa_forward must agree bit for bit). The oracle then recomputes, one
+by one, sampled parts of the result from inputs regenerated on the host from
+the same seeds: whole pyramid planes, the selections of sampled query blocks
+(bit-exact except near-ties), and the attention rows of sampled query blocks
+(on the GPU's own selection). The needle workload also checks that every
+planted needle block is selected for its target query block.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import gpu_util as gu
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _run(w, device):
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    shape = pisa.Shape.of(w)
+    q, k, v = (workloads.device_tensor(w, t, device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, device)
+    pyr = pisa.build_pyramid(shape, k)
+    idx = pisa.select_blocks(shape, q, pyr, ws)
+    o, lse = pisa.sparse_attention(shape, q, k, v, idx, ws)
+    o2, lse2, idx2 = pisa.forward(shape, q, k, v, pisa.new_workspace(shape, device), idx=True)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, w.name)
+    assert torch.equal(idx, idx2) and torch.equal(o, o2) and torch.equal(lse, lse2)
+    del q, k, v, o2, lse2, idx2
+    return shape, pyr, idx.cpu().numpy(), o, lse
+
+
+def _check_planes(w, shape, pyr, idx, o, lse, planes, n_sel, n_att, seed):
+    """Pyramid, selection and attention of sampled (batch, KV head) planes against the oracle."""
+    import block_sparse_long_pisa_b200 as pisa
+    _, offs = pisa.level_layout(shape)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    nqb = shape.n_qblocks
+    g = w.group
+    scale = 1.0 / math.sqrt(w.head_dim)
+    near_total = 0
+    for (b, kvh) in planes:
+        K = workloads.plane_f32(w, "k", b, kvh)
+        V = workloads.plane_f32(w, "v", b, kvh)
+        Qh = np.stack([workloads.plane_f32(w, "q", b, h) for h in range(kvh * g, (kvh + 1) * g)])
+        levels = oracle.build_pyramid(K, w.block, w.factor)
+        gu.assert_pyramid_close(gu.host_f32(pyr[b, kvh]), levels, offs)
+        qbar = oracle.query_summary(Qh, 1 if w.decode else w.block)
+        if w.decode:
+            blocks_sel = [0]
+        else:
+            extra = [i for (i, _) in workloads.needles(w, b, kvh)] if w.keys == "needle" else []
+            picks = rng.choice(nqb, size=min(n_sel, nqb), replace=False).tolist()
+            blocks_sel = sorted(set(picks) | {0, nqb - 1} | set(extra))
+        for i in blocks_sel:
+            last = i if (w.causal and not w.decode) else w.n_blocks - 1
+            r = oracle.select_blocks(qbar[i], levels, w.factor, w.topk, last)
+            ref = np.full(w.topk, -1, dtype=np.int32)
+            ref[:len(r["idx"])] = r["idx"]
+            if not np.array_equal(idx[b, kvh, i], ref):
+                assert r["margin"] < gu.NEAR_TIE, (w.name, b, kvh, i, r["margin"])
+                near_total += 1
+        att_blocks = blocks_sel if w.decode else sorted(rng.choice(blocks_sel, size=min(n_att, len(blocks_sel)),
+                                                                   replace=False).tolist())
+        for i in att_blocks:
+            rows = np.arange(1) if w.decode else np.arange(i * w.block, (i + 1) * w.block)
+            pos = np.full(1, w.seq_kv - 1) if w.decode else rows
+            sel = [int(j) for j in idx[b, kvh, i] if j >= 0]
+            for hh in range(g):
+                h = kvh * g + hh
+                ro, rl = oracle.attend(Qh[hh, rows], pos, K, V, sel, w.block, bool(w.causal) and not w.decode, scale)
+                go = o[b, h, rows[0]:rows[-1] + 1].float().cpu().numpy()
+                gl = lse[b, h, rows[0]:rows[-1] + 1].cpu().numpy()
+                gu.assert_output_close(go, ro, gl, rl, f"{w.name} b{b} h{h} i{i}")
+    return near_total
+
+
+def test_causal32k(cuda_device):
+    w = workloads.WORKLOADS["causal32k"]
+    shape, pyr, idx, o, lse = _run(w, cuda_device)
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (0, 9), (0, 15)], 24, 6, 1)
+
+
+def test_gqa128k_bench_configuration(cuda_device):
+    w = workloads.WORKLOADS["gqa128k"]
+    shape, pyr, idx, o, lse = _run(w, cuda_device)
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (0, 5)], 16, 6, 2)
+    # every planted needle block is selected for its target query block, in every KV head
+    for kvh in range(w.heads_kv):
+        for (i, j) in workloads.needles(w, 0, kvh):
+            assert j in idx[0, kvh, i], (kvh, i, j)
+
+
+def test_long1m(cuda_device):
+    w = workloads.WORKLOADS["long1m"]
+    shape, pyr, idx, o, lse = _run(w, cuda_device)
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 3)], 12, 4, 3)
+
+
+def test_decode128k(cuda_device):
+    w = workloads.WORKLOADS["decode128k"]
+    shape, pyr, idx, o, lse = _run(w, cuda_device)
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (17, 3), (63, 7)], 1, 1, 4)
