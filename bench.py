@@ -77,13 +77,20 @@ def rank_workload(w, rank: int):
 
 
 def max_over_ranks(value: float, world: int) -> float:
+    """Slowest rank's time: every rank contributes its own CUDA-event measurement."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    on_gpu = dist.get_backend() == "nccl"
+    t = torch.tensor([value], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_step_max: float) -> float:
+    """Weak scaling: every rank processes its own sequence; the job rate uses the slowest rank."""
+    return tokens_per_rank * world / (ms_step_max / 1e3)
 
 
 def barrier(world: int):
@@ -301,8 +308,7 @@ def run_gpu(args, world, rank, local):
     roof_s = pool_bytes / hbm + max(sel_bytes / hbm, sel_flops / (FP32_ALU_TFLOPS * 1e12)) + attn_flops / bf16
     attn_s = stage_ms[2] / 1e3
     achieved = attn_flops / attn_s / 1e12
-    tokens = w.batch * w.seq_q * world
-    value = tokens / (ms_step / 1e3)
+    value = whole_job_tokens_per_s(w.batch * w.seq_q, world, ms_step)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -426,7 +432,8 @@ def run_decode(args, world, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": "decode tokens/s (one query token per sequence, KV 131072)", "value": w.batch * world / (ms_step / 1e3),
+        "metric": "decode tokens/s (one query token per sequence, KV 131072)",
+        "value": whole_job_tokens_per_s(w.batch, world, ms_step),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded numpy, bf16 RNE)",

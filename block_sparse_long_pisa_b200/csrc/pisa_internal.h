@@ -11,6 +11,8 @@ namespace pisa {
 
 // Upper bound on any single pipeline wait inside a kernel (ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Suspend-time hint of one mbarrier wait attempt (ns); the bound above still applies.
+constexpr uint32_t kTryWaitHintNs = 1000000u;
 
 // Selected blocks per query block the prefill attention kernel holds on chip.
 constexpr int kMaxPrefillTopk = 256;
