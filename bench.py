@@ -47,14 +47,24 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profiled_traffic(kernel_file: str, source: str) -> float | None:
-    """dram bytes per launch recorded by an ncu capture summary (profiles/<file>), or None when
-    absent or when the kernel source has changed since the capture (sha256 prefix recorded there)."""
+def kernel_source_hash(sources) -> str:
     import hashlib
+    h = hashlib.sha256()
+    for src in sources:
+        h.update(open(os.path.join(ROOT, src), "rb").read())
+    return h.hexdigest()[:16]
+
+
+ATTN_SOURCES = ("block_sparse_long_pisa_b200/csrc/attn_prefill.cu", "block_sparse_long_pisa_b200/csrc/pisa_device.cuh")
+
+
+def profiled_traffic(kernel_file: str, sources) -> float | None:
+    """dram bytes per launch recorded by an ncu capture summary (profiles/<file>), or None when
+    absent or when the kernel sources have changed since the capture (sha256 prefix recorded there)."""
     p = os.path.join(ROOT, "profiles", kernel_file)
     if not os.path.exists(p):
         return None
-    sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    sha = kernel_source_hash(sources)
     fields = dict(line.split(":", 1) for line in open(p) if ":" in line and not line.startswith((" ", "|", "#")))
     if fields.get("source_sha256_16", "").strip() != sha:
         return None
@@ -336,7 +346,7 @@ def run_gpu(args, world, rank, local):
     if rank != 0:
         return
     cpu = oracle_sample(bench_workload(args)) if world == 1 and not args.no_cpu_baseline else None
-    traffic = profiled_traffic("attn_prefill_gqa128k.md", "block_sparse_long_pisa_b200/csrc/attn_prefill.cu")
+    traffic = profiled_traffic("attn_prefill_gqa128k.md", ATTN_SOURCES)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
