@@ -39,8 +39,9 @@
 // leaves TMEM.
 //
 // Softmax arithmetic: packed fp32 pair instructions (f32x2) for the
-// scale-and-subtract and the row sum, and the exponentials split between the
-// MUFU unit and a polynomial on the FMA pipes.
+// scale-and-subtract and the row sum, exponentials on the MUFU unit. (Moving a
+// share of them to a polynomial on the FMA pipes measured slower here: the
+// softmax is bound by instruction issue and latency, not by MUFU throughput.)
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -80,8 +81,6 @@ struct PrefillCfg {
 // Lazy rescale threshold (log2 units): the running max is kept until a new
 // row max exceeds it by this much, so probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f;
-// Pairs of scores k with k % kPolyMod == kPolyMod - 1 take the FMA-pipe exp2.
-constexpr int kPolyMod = 3;
 
 template <int D, int BLK, int NM>
 __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
@@ -336,12 +335,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
                     if (TRACK) xm = fmax3(xm, x0, x1);
-                    uint64_t e2;
-                    if (!MASKED && (kk % kPolyMod) == kPolyMod - 1) {
-                        e2 = exp2_poly_x2(x0, x1);
-                    } else {
-                        e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
-                    }
+                    const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
                     sum2[k & 1] = f2_add(sum2[k & 1], e2);
                     float e0, e1;
                     f2_unpack(e2, e0, e1);

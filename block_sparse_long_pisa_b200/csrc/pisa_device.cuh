@@ -289,29 +289,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// 2^x for a pair of floats on the FMA pipes instead of the MUFU unit, so that
-// the softmax can split its exponentials between the two. Cody-Waite range
-// reduction: x = j + f with j = round(x) (obtained by adding 1.5 * 2^23, which
-// leaves j in the low mantissa bits) and f in [-0.5, 0.5]; 2^f from a degree-3
-// polynomial fitted for minimum relative error on that interval (max relative
-// error 7.5e-5, far below the bf16 rounding of the probabilities); 2^j added
-// into the exponent field. x is clamped at -126 so the exponent stays normal;
-// callers only pass finite x <= 8 (masked keys never take this path).
-__device__ __forceinline__ uint64_t exp2_poly_x2(float a, float b) {
-    const uint64_t x = f2_pack(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
-    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
-    const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
-    uint64_t p = f2_fma(f2_pack(0.05517132207751274f, 0.05517132207751274f), f,
-                        f2_pack(0.24261054396629333f, 0.24261054396629333f));
-    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-    p = f2_fma(p, f, f2_pack(0.9999281167984009f, 0.9999281167984009f));
-    uint32_t tl, th, pl, ph;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(tl), "=r"(th) : "l"(t));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(pl), "=r"(ph) : "l"(p));
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(pl + (tl << 23)), "r"(ph + (th << 23)));
-    return r;
-}
-
 }  // namespace pisa
