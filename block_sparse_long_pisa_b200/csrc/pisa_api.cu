@@ -85,6 +85,10 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->ws_part = o;
     if (p->decode)
         o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->dec_splits * p->gsel * (p->D + 2) * sizeof(float));
+    p->dense_select = !p->decode && p->nqb >= kDenseSelectMinQBlocks;
+    p->ws_scores = o;
+    if (p->dense_select)
+        o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->nqb * p->total_nodes * sizeof(float));
     p->ws_total = o;
     return PISA_OK;
 }
@@ -156,7 +160,8 @@ static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cud
 }
 
 static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, const int32_t* budget,
-                          int32_t* idx, float* margin, uint32_t* status, cudaStream_t st) {
+                          int32_t* idx, float* margin, uint8_t* ws, cudaStream_t st) {
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws);
     SelectParams sp{};
     sp.qbar = qbar;
     sp.pyr = pyr;
@@ -183,8 +188,8 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
         sp.width[l] = w;
         w = w > (int64_t(1) << 40) ? w : w * pl.f;
     }
-    if (!launch_select(sp, pl.B, st)) return PISA_ERR_CUDA;
-    ++g_launches;
+    sp.scores = pl.dense_select ? reinterpret_cast<float*>(ws + pl.ws_scores) : nullptr;
+    if (!launch_select(sp, pl.B, st, &g_launches)) return PISA_ERR_CUDA;
     return PISA_OK;
 }
 
@@ -319,7 +324,7 @@ pisa_status pisa_select_blocks(const pisa_shape* shape, const void* Q, const flo
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
     if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
-    return select(pl, qbar, pyramid, level_budget, idx, margin, reinterpret_cast<uint32_t*>(w), st);
+    return select(pl, qbar, pyramid, level_budget, idx, margin, w, st);
 }
 
 pisa_status pisa_sparse_attention(const pisa_shape* shape, const void* Q, const void* K, const void* V,
@@ -353,7 +358,7 @@ pisa_status pisa_forward(const pisa_shape* shape, const void* Q, const void* K, 
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + pl.ws_idx);
     if ((s = build_pyramid(pl, K, pyr, st)) != PISA_OK) return s;
     if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
-    if ((s = select(pl, qbar, pyr, nullptr, idx, nullptr, reinterpret_cast<uint32_t*>(w), st)) != PISA_OK) return s;
+    if ((s = select(pl, qbar, pyr, nullptr, idx, nullptr, w, st)) != PISA_OK) return s;
     return attention(pl, Q, K, V, idx, O, lse, w, st);
 }
 

@@ -16,6 +16,10 @@ constexpr uint32_t kTryWaitHintNs = 1000000u;
 
 // Selected blocks per query block the prefill attention kernel holds on chip.
 constexpr int kMaxPrefillTopk = 256;
+// Prefill with at least this many query blocks per selection row scores every
+// eligible node densely (the tiles are shared by 128 query blocks); fewer
+// query blocks (and decode) score only the descent's candidates.
+constexpr int kDenseSelectMinQBlocks = 16;
 
 // Bytes reserved for the status word at the start of the workspace.
 constexpr size_t kStatusBytes = 256;
@@ -44,7 +48,8 @@ struct Plan {
     int32_t dec_bps;     // selected blocks per split
     int32_t dec_splits;
     // workspace layout (byte offsets)
-    size_t ws_pyramid, ws_qbar, ws_idx, ws_part, ws_total;
+    size_t ws_pyramid, ws_qbar, ws_idx, ws_part, ws_scores, ws_total;
+    int32_t dense_select;       // prefill selection scores densely (score plane in the workspace)
     size_t pyramid_bytes;
 };
 
@@ -86,6 +91,9 @@ struct SelectParams {
     int32_t loff[PISA_MAX_LEVELS];
     int32_t budget[PISA_MAX_LEVELS];
     int64_t width[PISA_MAX_LEVELS];  // f^l (saturated)
+    float* scores;                   // dense prefill scoring: fp32 [B, Hsel, nqb, total_nodes], or null
+    int32_t tile_off[PISA_MAX_LEVELS + 1];  // score tiles before level l (set by the launcher)
+    int32_t tiles_c[PISA_MAX_LEVELS];       // node tiles of level l (set by the launcher)
 };
 
 struct AttnParams {
@@ -116,7 +124,12 @@ struct DecodeParams {
 
 bool launch_block_mean(const MeanParams& p, cudaStream_t st);
 bool launch_pyramid_level(const LevelParams& p, cudaStream_t st);
-bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st);
+// Launches the selection; adds the kernels it launched to *launches. Prefill
+// with a score plane and candidate sets of at most 1024 runs the dense scoring
+// kernel and the warp descent; otherwise the one-CTA-per-row sparse descent.
+bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
+int dense_select_cap(int cap);
+bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st);
 // Prefill attention: builds the tensor maps and picks the kernel variant.
 pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
                                 cudaStream_t st, int32_t* launches);

@@ -26,6 +26,8 @@
 namespace pisa {
 
 constexpr int kSelThreads = 128;
+// Candidates one group of eight lanes scores per loop trip (all their loads are issued first).
+constexpr int kSelBatch = 4;
 
 __device__ __forceinline__ uint32_t order_bits(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -115,8 +117,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
         for (int l = 1; l < p.L; ++l) {
             const int64_t wl = p.width[l], wb = p.width[l - 1];
             const int64_t c_l = last / wl, c_b = last / wb;
-            for (int64_t c = c_l * p.factor; c < c_b; ++c)
-                sum += static_cast<float>(wb) * plane[(p.loff[l - 1] + c) * D + d];
+            // at most f-1 full children precede the straddling one; load them together
+            float ch[8];
+            const int nch = static_cast<int>(c_b - c_l * p.factor);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                ch[u] = u < nch ? plane[(p.loff[l - 1] + c_l * p.factor + u) * D + d] : 0.f;
+            for (int u = 8; u < nch; ++u) sum += static_cast<float>(wb) * plane[(p.loff[l - 1] + c_l * p.factor + u) * D + d];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (u < nch) sum += static_cast<float>(wb) * ch[u];
             part[l * D + d] = sum / static_cast<float>(last - c_l * wl + 1);
         }
     }
@@ -153,28 +163,41 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             const int n = next_pow2(ncand);
             const int64_t c_part = last / p.width[l];
             const bool has_part = min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
-            // 8 lanes per candidate: each warp load instruction covers four whole 128-byte lines
-            for (int t0 = 0; t0 < n; t0 += kSelThreads / 8) {
-                const int t = t0 + (tid >> 3);
-                const bool live = t < ncand && cand[t] >= 0;
-                const int32_t c = live ? cand[t] : 0;
-                float acc = 0.f;
-                if (live) {
-                    const float* v = (has_part && c == c_part) ? part + l * D
-                                                               : plane + static_cast<int64_t>(p.loff[l] + c) * D;
+            // 8 lanes per candidate: each warp load instruction covers four whole 128-byte lines;
+            // each group issues the loads of kSelBatch candidates before any arithmetic
+            constexpr int GROUPS = kSelThreads / 8;
+            for (int t0 = 0; t0 < n; t0 += GROUPS * kSelBatch) {
+                float4 x[kSelBatch][D / 32];
+                int32_t cb[kSelBatch];
+                bool live[kSelBatch];
+#pragma unroll
+                for (int j = 0; j < kSelBatch; ++j) {
+                    const int t = t0 + j * GROUPS + (tid >> 3);
+                    live[j] = t < ncand && cand[t] >= 0;
+                    cb[j] = live[j] ? cand[t] : 0;
+                    const float* v = (has_part && cb[j] == c_part) ? part + l * D
+                                                                  : plane + static_cast<int64_t>(p.loff[l] + cb[j]) * D;
+#pragma unroll
+                    for (int k = 0; k < D / 32; ++k)
+                        x[j][k] = live[j] ? *reinterpret_cast<const float4*>(v + 32 * k + 4 * sub)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < kSelBatch; ++j) {
+                    float acc = 0.f;
 #pragma unroll
                     for (int k = 0; k < D / 32; ++k) {
-                        const float4 x = *reinterpret_cast<const float4*>(v + 32 * k + 4 * sub);
-                        acc = fmaf(qv[k].x, x.x, acc);
-                        acc = fmaf(qv[k].y, x.y, acc);
-                        acc = fmaf(qv[k].z, x.z, acc);
-                        acc = fmaf(qv[k].w, x.w, acc);
+                        acc = fmaf(qv[k].x, x[j][k].x, acc);
+                        acc = fmaf(qv[k].y, x[j][k].y, acc);
+                        acc = fmaf(qv[k].z, x[j][k].z, acc);
+                        acc = fmaf(qv[k].w, x[j][k].w, acc);
                     }
+                    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
+                    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+                    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+                    const int t = t0 + j * GROUPS + (tid >> 3);
+                    if (sub == 0 && t < n) keys[t] = live[j] ? rank_key(acc, cb[j]) : 0ull;
                 }
-                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
-                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
-                acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
-                if (sub == 0 && t < n) keys[t] = live ? rank_key(acc, c) : 0ull;
             }
             __syncthreads();
             const int nvalid = s_nvalid;
@@ -219,12 +242,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     if (p.margin != nullptr && tid == 0) p.margin[row] = s_margin;
 }
 
-bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st) {
+bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_t* launches) {
     int maxb = 1;
     for (int l = 0; l < p.L; ++l) maxb = max(maxb, p.budget[l]);
     int cap = 1;
     while (cap < max(p.factor * maxb, p.lsize[p.L - 1])) cap <<= 1;
     if (cap < 4) cap = 4;  // keeps the fp32 query row 16-byte aligned
+    if (p.scores != nullptr && !p.decode && dense_select_cap(cap) > 0) {
+        *launches += 2;
+        return launch_select_dense(p, batch, cap, st);
+    }
+    *launches += 1;
     const size_t smem = static_cast<size_t>(cap) * (sizeof(uint64_t) + sizeof(int32_t)) +
                         static_cast<size_t>(p.D) * (1 + p.L) * sizeof(float);
     dim3 grid(p.nqb, p.Hsel, batch);

@@ -102,6 +102,9 @@ PISA_API pisa_status pisa_pyramid_size(const pisa_shape *shape, size_t *bytes);
  * pisa_sparse_attention need for this shape (one size serves all three).
  * The first 256 bytes are the device status word; zero them once when the
  * workspace is allocated (pisa_check_status clears them after each read).
+ * Prefill with 16 or more query blocks also holds an fp32 score plane of
+ * B * Hsel * (Nq / b) * total_nodes values (Hsel = heads_kv, or heads_q with
+ * select_per_qhead), used by the selection.
  * Host only. */
 PISA_API pisa_status pisa_workspace_size(const pisa_shape *shape, size_t *bytes);
 

@@ -27,6 +27,8 @@ SMALL = {
                                  "clustered", 16),
     "gqa4-d64-noncausal": W("gqa4-d64-noncausal", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 5, 0, "iid", 17),
     "gqa4-needle": W("gqa4-needle", 1, 8, 2, 256 * 64, 256 * 64, 128, 64, 4, 16, 1, "needle", 18),
+    # fewer query blocks than the dense-scoring threshold: the sparse descent runs for prefill
+    "gqa4-causal-short": W("gqa4-causal-short", 2, 8, 2, 13 * 64, 13 * 64, 128, 64, 4, 3, 1, "iid", 23),
     "decode-gqa4": W("decode-gqa4", 3, 8, 2, 1, 45 * 64, 128, 64, 4, 9, 0, "clustered", 19),
     "decode-d64-b128": W("decode-d64-b128", 2, 4, 4, 1, 40 * 128, 64, 128, 8, 6, 0, "iid", 20),
 }
