@@ -371,8 +371,8 @@ def run_gpu(args, world, rank, local):
 
 def bench_workload(args):
     w = workloads.WORKLOADS[args.workload]
-    if args.seq:
-        w = w.replace(seq_q=args.seq, seq_kv=args.seq, name=f"{w.name}@N={args.seq}")
+    if args.seq:  # decode keeps its single query token
+        w = w.replace(seq_q=1 if w.decode else args.seq, seq_kv=args.seq, name=f"{w.name}@N={args.seq}")
     return w
 
 

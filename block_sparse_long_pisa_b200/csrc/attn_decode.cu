@@ -1,17 +1,20 @@
 // Decode: one query token per sequence at position N-1 attends to the K/V
 // blocks its pyramid descent selected. The work is bound by the bytes of the
-// selected K/V blocks, so the kernel is built for HBM streaming, not the
-// tensor core:
+// selected K/V blocks; the arithmetic only has to stay out of the way:
 //
-//   attn_decode_kernel: one CTA per (batch, selection row, split). A split is
-//     up to `bps` consecutive entries of the selected-block list. Each K or V
-//     block (b rows x D, contiguous in memory) is fetched by one bulk copy
-//     into a double-buffered shared-memory ring. The CTA's gh query heads run
-//     an online softmax over the split's keys with fp32 FMA and leave an
-//     unnormalised partial (o, running max m, sum l) in the workspace.
+//   attn_decode_kernel: one CTA of four warps per (batch, selection row,
+//     split); a split is up to `bps` consecutive entries of the compacted
+//     block list. K and V blocks arrive by 2-D TMA (128-byte swizzle) in a
+//     ring of NSTG stages. The gh <= 8 query heads of the selection row are
+//     the rows of a 16-row bf16 tensor-core tile (rows gh.. are zero): each
+//     warp takes a quarter of every block's keys and computes its scores and
+//     its share of P.V with mma.sync m16n8k16 (fragments by ldmatrix from the
+//     swizzled tiles), with its own online softmax. At the end the four warps'
+//     (o, m, l) combine into one unnormalised partial per head.
 //   attn_merge_kernel: combines the partials of all splits with the
 //     online-softmax merge of the Pulsar Attention page ("Phase 2"):
 //     m = max m_s, l = sum exp2(m_s - m) l_s, o = sum exp2(m_s - m) o_s / l.
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "pisa_device.cuh"
@@ -21,18 +24,51 @@ namespace pisa {
 constexpr int kDecThreads = 128;
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const DecodeParams p) {
-    constexpr int TILE = BLK * D * 2;  // bytes of one K (or V) block
-    extern __shared__ __align__(1024) uint8_t sm[];
-    uint8_t* kbuf = sm;                          // [2][TILE]
-    uint8_t* vbuf = sm + 2 * TILE;               // [2][TILE]
-    float* qs = reinterpret_cast<float*>(sm + 4 * TILE);  // [gh][D], pre-scaled by scale*log2(e)
-    float* ss = qs + 8 * D;                      // [gh][BLK] scores, then probabilities
-    float* m_run = ss + 8 * BLK;                 // [gh]
-    float* l_run = m_run + 8;                    // [gh]
-    float* alpha = l_run + 8;                    // [gh]
-    int32_t* list = reinterpret_cast<int32_t*>(alpha + 8);  // this split's blocks
-    __shared__ __align__(8) uint64_t full[2];
+struct DecodeCfg {
+    static constexpr int DS = D / 64;                      // 128-byte column tiles of a row
+    static constexpr int SUBT = BLK * 128;                 // one [BLK rows x 128 B] swizzled tile
+    static constexpr int TILE = DS * SUBT;                 // one K (or V) block
+    static constexpr int STAGE = 2 * TILE;                 // K and V
+    static constexpr int NSTG = STAGE <= 16384 ? 4 : (STAGE <= 32768 ? 3 : 2);
+    static constexpr int KW = BLK / 4;                     // keys of a block per warp
+    static constexpr int NT = KW / 8;                      // score n-tiles per warp
+    static constexpr int COMBINE = 4 * 8 * (D + 2) * 4;    // per-warp (o, m, l) of 8 heads
+    static constexpr int SMEM = 1024 + NSTG * STAGE;
+    static_assert(COMBINE <= NSTG * STAGE, "combine area reuses the ring");
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D += A B for one m16n8k16 bf16 tile with fp32 accumulators; a1 = a3 = 0 (rows 8-15 unused)
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// byte offset of row `row`, 16-byte chunk `chunk` (of the 8 in a 128-byte row) inside a swizzled tile
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+    return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                  const __grid_constant__ CUtensorMap tmV,
+                                                                  const DecodeParams p) {
+    using C = DecodeCfg<D, BLK>;
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[C::NSTG], empty[C::NSTG];
+    __shared__ int32_t list[kDecMaxBps];
     __shared__ int s_cnt;
 
     const int split = blockIdx.x, hs = blockIdx.y, b = blockIdx.z;
@@ -46,7 +82,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const DecodePa
     if (warp == 0) {
         const int32_t* row = p.idx + (static_cast<int64_t>(b) * p.Hsel + hs) * p.topk;
         const int lo = split * p.bps, hi = lo + p.bps;
-        int cnt = 0, taken = 0;
+        int cnt = 0;
         for (int t0 = 0; t0 < p.topk; t0 += 32) {
             const int t = t0 + lane;
             const int32_t j = t < p.topk ? row[t] : -1;
@@ -58,148 +94,166 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const DecodePa
             if (ok && pos >= lo && pos < hi) list[pos - lo] = j;
             cnt += __popc(m);
         }
-        taken = min(max(cnt - lo, 0), p.bps);
         if (lane == 0) {
-            s_cnt = taken;
-            mbar_init(&full[0], 1);
-            mbar_init(&full[1], 1);
+            s_cnt = min(max(cnt - lo, 0), p.bps);
+            for (int s = 0; s < C::NSTG; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 4);
+            }
             fence_barrier_init();
         }
     }
-    const float cs = p.scale_log2;
-    for (int e = tid; e < gh * D; e += kDecThreads) {
-        const int hh = e / D, d = e % D;
-        qs[hh * D + d] = __bfloat162float(p.Q[(static_cast<int64_t>(b) * p.Hq + head0 + hh) * D + d]) * cs;
-    }
-    if (tid < gh) {
-        m_run[tid] = -INFINITY;
-        l_run[tid] = 0.f;
-    }
     __syncthreads();
     const int cnt = s_cnt;
-    const __nv_bfloat16* kplane = p.K + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N * D;
-    const __nv_bfloat16* vplane = p.V + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N * D;
+    const int64_t row0 = (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N;  // first K/V row of this plane
+    auto issue = [&](int n) {
+        const int s = n % C::NSTG;
+        uint8_t* kt = ring + s * C::STAGE;
+        mbar_arrive_expect_tx(&full[s], C::STAGE);
+        const int y = static_cast<int>(row0 + static_cast<int64_t>(list[n]) * BLK);
+#pragma unroll
+        for (int c = 0; c < C::DS; ++c) {
+            tma_load_2d(kt + c * C::SUBT, &tmK, c * 64, y, &full[s]);
+            tma_load_2d(kt + C::TILE + c * C::SUBT, &tmV, c * 64, y, &full[s]);
+        }
+    };
     int issued = 0;  // thread 0: blocks whose copies were started
     if (tid == 0) {
-        for (int u = 0; u < 2 && u < cnt; ++u, ++issued) {
-            mbar_arrive_expect_tx(&full[u], 2 * TILE);
-            bulk_load(kbuf + u * TILE, kplane + static_cast<int64_t>(list[u]) * BLK * D, TILE, &full[u]);
-            bulk_load(vbuf + u * TILE, vplane + static_cast<int64_t>(list[u]) * BLK * D, TILE, &full[u]);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        for (; issued < C::NSTG && issued < cnt; ++issued) issue(issued);
+    }
+
+    // query fragments: row hh = lane / 4 (zero past gh), dims 16 ks + 2 (lane % 4) (+8)
+    const int hh = lane >> 2, q4 = lane & 3;
+    uint32_t qa[D / 16][2];
+    {
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.Q + (static_cast<int64_t>(b) * p.Hq + head0 + hh) * D);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            qa[ks][0] = hh < gh ? qrow[ks * 8 + q4] : 0u;
+            qa[ks][1] = hh < gh ? qrow[ks * 8 + 4 + q4] : 0u;
         }
     }
-    // output accumulators: this thread owns (head, 4 dims) chunks e = tid + 128 * u
-    constexpr int CHUNKS = D / 4;
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const float cs = p.scale_log2;
+    float o[D / 8][4];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m_run = -INFINITY, l_thr = 0.f;  // this thread's row hh: running max, partial sum
+    const int kw0 = warp * C::KW;          // this warp's keys of every block
+    const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix and row this lane addresses
     bool ok = true;
     int n = 0;
     for (; n < cnt; ++n) {
-        const int buf = n & 1;
-        ok = mbar_wait(&full[buf], (n >> 1) & 1, p.status, detail_base | 0x01u);
-        if (!__syncthreads_and(ok)) {
-            ok = false;
-            break;
-        }
-        const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(kbuf + buf * TILE);
-        const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(vbuf + buf * TILE);
-        // scores: pair e -> (head e / BLK, key e % BLK); rotate the 16-byte chunk order per key
-        for (int e = tid; e < gh * BLK; e += kDecThreads) {
-            const int hh = e / BLK, key = e % BLK;
-            const uint4* krow = reinterpret_cast<const uint4*>(kt + key * D);
-            const float* q = qs + hh * D;
-            float a = 0.f;
-#pragma unroll 4
-            for (int cc = 0; cc < D / 8; ++cc) {
-                const int c = (cc + key) & (D / 8 - 1);
-                const uint4 v = krow[c];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const int s = n % C::NSTG;
+        ok = mbar_wait(&full[s], (n / C::NSTG) & 1, p.status, detail_base | 0x01u);
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        const uint32_t kbase = smem_u32(ring + s * C::STAGE), vbase = kbase + C::TILE;
+        // scores of this warp's keys: S[hh][key] for key = kw0 + 8 nt + 2 (lane % 4) (+1)
+        float sc[C::NT][4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    a = fmaf(q[c * 8 + 2 * k], __uint_as_float(w[k] << 16), a);
-                    a = fmaf(q[c * 8 + 2 * k + 1], __uint_as_float(w[k] & 0xFFFF0000u), a);
-                }
-            }
-            ss[hh * BLK + key] = a;
-        }
-        __syncthreads();
-        // online softmax statistics, one warp per head
-        for (int hh = warp; hh < gh; hh += kDecThreads / 32) {
-            float mx = -INFINITY;
-            for (int key = lane; key < BLK; key += 32) mx = fmaxf(mx, ss[hh * BLK + key]);
+        for (int nt = 0; nt < C::NT; ++nt) {
+            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+            const int key = kw0 + 8 * nt + mr;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-            const float m_old = m_run[hh];
-            const float m_new = fmaxf(m_old, mx);
-            float sum = 0.f;
-            for (int key = lane; key < BLK; key += 32) {
-                const float e2 = fast_exp2(ss[hh * BLK + key] - m_new);
-                ss[hh * BLK + key] = e2;
-                sum += e2;
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-            __syncwarp();
-            if (lane == 0) {
-                const float a = fast_exp2(m_old - m_new);
-                alpha[hh] = a;
-                l_run[hh] = l_run[hh] * a + sum;
-                m_run[hh] = m_new;
+            for (int j = 0; j < D / 32; ++j) {  // two k-steps (32 dims) per ldmatrix.x4
+                const int dim = 32 * j + 8 * mi;
+                uint32_t kb[4];
+                ldsm_x4(kbase + (dim / 64) * C::SUBT + sw128(key, (dim % 64) / 8), kb);
+                mma_16816(sc[nt], qa[2 * j][0], qa[2 * j][1], kb[0], kb[1]);
+                mma_16816(sc[nt], qa[2 * j + 1][0], qa[2 * j + 1][1], kb[2], kb[3]);
             }
         }
-        __syncthreads();
-        // o = o * alpha + P V
+        // online softmax of row hh over this warp's keys (the four lanes of a quad share the row)
+        float mx = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + kDecThreads * u;
-            if (e < gh * CHUNKS) {
-                const int hh = e / CHUNKS, dq = e % CHUNKS;
-                const float a = alpha[hh];
-                float o0 = acc[u][0] * a, o1 = acc[u][1] * a, o2 = acc[u][2] * a, o3 = acc[u][3] * a;
-                const float* pr = ss + hh * BLK;
-#pragma unroll 4
-                for (int key = 0; key < BLK; ++key) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(vt + key * D + dq * 4);
-                    const float pk = pr[key];
-                    o0 = fmaf(pk, __uint_as_float(v.x << 16), o0);
-                    o1 = fmaf(pk, __uint_as_float(v.x & 0xFFFF0000u), o1);
-                    o2 = fmaf(pk, __uint_as_float(v.y << 16), o2);
-                    o3 = fmaf(pk, __uint_as_float(v.y & 0xFFFF0000u), o3);
-                }
-                acc[u][0] = o0;
-                acc[u][1] = o1;
-                acc[u][2] = o2;
-                acc[u][3] = o3;
+        for (int nt = 0; nt < C::NT; ++nt) {
+            sc[nt][0] *= cs;
+            sc[nt][1] *= cs;
+            mx = fmax3(mx, sc[nt][0], sc[nt][1]);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = fast_exp2(m_run - m_new);
+        m_run = m_new;
+        l_thr *= alpha;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+            o[j][0] *= alpha;
+            o[j][1] *= alpha;
+        }
+        uint32_t pa[C::NT];  // P as bf16 pairs, A-fragment halves
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+            const float e0 = fast_exp2(sc[nt][0] - m_new), e1 = fast_exp2(sc[nt][1] - m_new);
+            l_thr += e0 + e1;
+            pa[nt] = pack_bf16x2(e0, e1);
+        }
+        // O[hh][:] += P V over this warp's keys: k-steps of 16 keys, two n-tiles per ldmatrix.x4
+#pragma unroll
+        for (int kk = 0; kk < C::KW / 16; ++kk) {
+            const int key = kw0 + 16 * kk + mr + 8 * (mi & 1);
+#pragma unroll
+            for (int jj = 0; jj < D / 16; ++jj) {
+                const int dim = 16 * jj + 8 * (mi >> 1);
+                uint32_t vb[4];
+                ldsm_x4_t(vbase + (dim / 64) * C::SUBT + sw128(key, (dim % 64) / 8), vb);
+                mma_16816(o[2 * jj], pa[2 * kk], pa[2 * kk + 1], vb[0], vb[1]);
+                mma_16816(o[2 * jj + 1], pa[2 * kk], pa[2 * kk + 1], vb[2], vb[3]);
             }
         }
-        __syncthreads();
-        // refill this buffer with block n + 2
-        if (tid == 0 && n + 2 < cnt) {
-            ++issued;
-            mbar_arrive_expect_tx(&full[buf], 2 * TILE);
-            bulk_load(kbuf + buf * TILE, kplane + static_cast<int64_t>(list[n + 2]) * BLK * D, TILE, &full[buf]);
-            bulk_load(vbuf + buf * TILE, vplane + static_cast<int64_t>(list[n + 2]) * BLK * D, TILE, &full[buf]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        // refill this stage with block n + NSTG once all four warps are done with it
+        if (tid == 0 && n + C::NSTG < cnt) {
+            if (!mbar_wait(&empty[s], (n / C::NSTG) & 1, p.status, detail_base | 0x03u)) ok = false;
+            else {
+                issue(n + C::NSTG);
+                ++issued;
+            }
         }
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
     }
-    // partial: [gh][D] o, then m, l
-    float* part = p.part + ((static_cast<int64_t>(b) * p.Hsel + hs) * p.splits + split) * gh * (D + 2);
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int e = tid + kDecThreads * u;
-        if (e < gh * CHUNKS) {
-            const int hh = e / CHUNKS, dq = e % CHUNKS;
-            float* dst = part + hh * (D + 2) + dq * 4;
-            dst[0] = acc[u][0];
-            dst[1] = acc[u][1];
-            dst[2] = acc[u][2];
-            dst[3] = acc[u][3];
-        }
-    }
-    if (tid < gh) {
-        part[tid * (D + 2) + D] = (ok && cnt > 0) ? m_run[tid] : -INFINITY;
-        part[tid * (D + 2) + D + 1] = (ok && cnt > 0) ? l_run[tid] : 0.f;
-    }
-    // in-flight copies land before the CTA exits (only after a failed wait can any be pending)
+    // in-flight copies land before the ring is reused (only after a failed wait can any be pending)
     if (tid == 0 && !ok) {
-        for (int u = n; u < issued; ++u) mbar_wait(&full[u & 1], (u >> 1) & 1, p.status, detail_base | 0x02u);
+        for (int u = n; u < issued; ++u) mbar_wait(&full[u % C::NSTG], (u / C::NSTG) & 1, p.status, detail_base | 0x02u);
+    }
+    const bool all_ok = __syncthreads_and(ok);
+    // the four warps' (o, m, l) of heads 0..gh-1 meet in the ring, then one partial per head
+    float* cw = reinterpret_cast<float*>(ring);  // [warp][head][D + 2]
+    l_thr += __shfl_xor_sync(0xFFFFFFFFu, l_thr, 1);
+    l_thr += __shfl_xor_sync(0xFFFFFFFFu, l_thr, 2);
+    if (hh < gh) {
+        float* dst = cw + (warp * 8 + hh) * (D + 2);
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+            dst[8 * j + 2 * q4] = o[j][0];
+            dst[8 * j + 2 * q4 + 1] = o[j][1];
+        }
+        if (q4 == 0) {
+            dst[D] = (all_ok && cnt > 0) ? m_run : -INFINITY;
+            dst[D + 1] = l_thr;
+        }
+    }
+    __syncthreads();
+    float* part = p.part + ((static_cast<int64_t>(b) * p.Hsel + hs) * p.splits + split) * gh * (D + 2);
+    for (int e = tid; e < gh * (D + 2); e += kDecThreads) {
+        const int h2 = e / (D + 2), d = e % (D + 2);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, cw[(w * 8 + h2) * (D + 2) + D]);
+        float v = 0.f;
+        if (d == D) {
+            v = M;
+        } else if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float* src = cw + (w * 8 + h2) * (D + 2);
+                v += fast_exp2(src[D] - M) * src[d == D + 1 ? D + 1 : d];
+            }
+        }
+        part[h2 * (D + 2) + d] = v;
     }
 }
 
@@ -229,15 +283,18 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const DecodeParams p) {
 
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches) {
     const int D = pl.D, BLK = pl.blk;
-    const size_t tile = static_cast<size_t>(BLK) * D * 2;
-    const size_t smem = 4 * tile + (8 * D + 8 * BLK + 24) * sizeof(float) + static_cast<size_t>(p.bps) * 4;
+    const int64_t krows = static_cast<int64_t>(pl.B) * pl.Hkv * pl.N;
+    if (krows > INT32_MAX) return false;
+    CUtensorMap tk, tv;
+    if (!make_tmap_2d(&tk, p.K, krows, D, BLK) || !make_tmap_2d(&tv, p.V, krows, D, BLK)) return false;
     dim3 grid(p.splits, p.Hsel, pl.B);
     cudaError_t e = cudaSuccess;
 #define PISA_DECODE_CASE(DD, BB)                                                                              \
     if (D == DD && BLK == BB) {                                                                               \
         e = cudaFuncSetAttribute(attn_decode_kernel<DD, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
-                                 static_cast<int>(smem));                                                    \
-        if (e == cudaSuccess) attn_decode_kernel<DD, BB><<<grid, kDecThreads, smem, st>>>(p);                \
+                                 DecodeCfg<DD, BB>::SMEM);                                                    \
+        if (e == cudaSuccess)                                                                                 \
+            attn_decode_kernel<DD, BB><<<grid, kDecThreads, DecodeCfg<DD, BB>::SMEM, st>>>(tk, tv, p);        \
     }
     PISA_DECODE_CASE(64, 64)
     PISA_DECODE_CASE(64, 128)

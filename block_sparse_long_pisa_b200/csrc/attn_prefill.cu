@@ -513,7 +513,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2-D view [rows, D] of a bf16 [.., tokens, D] tensor; boxes of 64 columns x box_rows rows, 128-byte swizzle.
-static bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows) {
+bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (enc == nullptr) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
@@ -545,8 +545,8 @@ pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, co
     CUtensorMap tq, tk, tv;
     const int64_t qrows = static_cast<int64_t>(pl.B) * pl.Hq * pl.N;
     const int64_t krows = static_cast<int64_t>(pl.B) * pl.Hkv * pl.N;
-    if (!make_tmap(&tq, Q, qrows, pl.D, pl.blk) || !make_tmap(&tk, K, krows, pl.D, pl.blk) ||
-        !make_tmap(&tv, V, krows, pl.D, pl.blk))
+    if (!make_tmap_2d(&tq, Q, qrows, pl.D, pl.blk) || !make_tmap_2d(&tk, K, krows, pl.D, pl.blk) ||
+        !make_tmap_2d(&tv, V, krows, pl.D, pl.blk))
         return PISA_ERR_CUDA;
     const int nm = p.gh * pl.blk > 128 ? 2 : 1;
     dim3 grid(pl.nqb, pl.Hsel * p.chunks, pl.B);

@@ -71,7 +71,14 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     if (p->decode && p->gsel > 8) return PISA_ERR_UNSUPPORTED;
     if (!p->decode && p->topk > kMaxPrefillTopk) return PISA_ERR_UNSUPPORTED;
 
-    p->dec_bps = 4;
+    // decode split: enough CTAs to fill the 148 SMs about four times over, at most kDecMaxBps
+    // blocks per CTA (longer splits keep the copy ring streaming), at least 2
+    {
+        const int64_t rows = static_cast<int64_t>(p->B) * p->Hsel;
+        const int64_t want = (4 * 148 + rows - 1) / rows;  // splits per row wanted
+        const int64_t bps = (p->topk + want - 1) / want;
+        p->dec_bps = static_cast<int32_t>(bps < 2 ? 2 : (bps > kDecMaxBps ? kDecMaxBps : bps));
+    }
     p->dec_splits = p->decode ? (p->topk + p->dec_bps - 1) / p->dec_bps : 0;
 
     p->pyramid_bytes = static_cast<size_t>(p->B) * p->Hkv * p->total_nodes * p->D * sizeof(float);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "pisa.h"
 
 namespace pisa {
@@ -16,6 +18,8 @@ constexpr uint32_t kTryWaitHintNs = 1000000u;
 
 // Selected blocks per query block the prefill attention kernel holds on chip.
 constexpr int kMaxPrefillTopk = 256;
+// Largest number of selected blocks one decode CTA streams (its block list lives in shared memory).
+constexpr int kDecMaxBps = 16;
 // Prefill with at least this many query blocks per selection row scores every
 // eligible node densely (the tiles are shared by 128 query blocks); fewer
 // query blocks (and decode) score only the descent's candidates.
@@ -134,5 +138,7 @@ bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st
 pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
                                 cudaStream_t st, int32_t* launches);
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
+// 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
 
 }  // namespace pisa
