@@ -18,7 +18,7 @@
 //                      lanes 32*(w%4).. of tile (w/4)%NM and owns the 64
 //                      score columns of its half (w/(4*NM)); the partner warp
 //                      of the other half shares the rows. They exchange row
-//                      maxima and sums through shared memory and a 64-thread
+//                      maxima and sums through a TMEM column and a 64-thread
 //                      named barrier, and each writes half of O at the end.
 //   warp 8*NM          producer: lane 0 streams K groups, lane 1 V groups, by
 //                      2-D TMA into NST-deep rings (each with its own empty
@@ -59,8 +59,7 @@ struct PrefillCfg {
     static constexpr int Q_BYTES = NM * DS * SUB;
     static constexpr int KG_BYTES = DS * SUB;          // a 128-key K (or V) group
     static constexpr int MAX_LIST = kMaxPrefillTopk;   // selected blocks per query block
-    static constexpr int XCH = 2 * 2 * NM * 128 * 4;       // [parity][half][tile][row] row statistics
-    static constexpr int AUX = 512 + MAX_LIST * 4 + XCH;   // barriers, TMEM slot, block list, exchange
+    static constexpr int AUX = 512 + MAX_LIST * 4;         // barriers, TMEM slot, block list
     static constexpr int SMEM_LIMIT = 232448;          // 227 KB opt-in maximum
     static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - Q_BYTES - AUX) / (2 * KG_BYTES);
     static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
@@ -76,6 +75,7 @@ struct PrefillCfg {
     static_assert(NST >= 2, "shared memory too small for double-buffered K/V rings");
     static_assert(TMEM_NEED <= 512, "TMEM budget exceeded");
     static_assert(BLK == 64 || BLK == 128, "key block of 64 or 128");
+    static_assert(SMEM < (1 << 18), "descriptor offsets assume shared addresses below 2^18");
 };
 
 // Lazy rescale threshold (log2 units): the running max is kept until a new
@@ -102,12 +102,11 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     uint64_t* s_full = v_empty + C::NST;      // NM   (S of tile h in TMEM)
     uint64_t* p_full = s_full + NM;           // NM   (P of tile h in TMEM, O rescaled)
     uint64_t* pv_done = p_full + NM;          // NM   (P.V of tile h completed)
-    uint64_t* x_bar = pv_done + NM;           // 4*NM (two softmax warps of a row quadrant meet)
-    uint64_t* mma_final = x_bar + 4 * NM;     // 1
+    uint64_t* mma_final = pv_done + NM;       // 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
     int32_t* s_nsel = reinterpret_cast<int32_t*>(tmem_slot + 1);
+    int32_t* s_diag = s_nsel + 1;             // list position of the diagonal block i, -1 if absent
     int32_t* list = reinterpret_cast<int32_t*>(aux + 512);
-    float* xch = reinterpret_cast<float*>(aux + 512 + C::MAX_LIST * 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -133,7 +132,6 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             mbar_init(p_full + h, 256);
             mbar_init(pv_done + h, 1);
         }
-        for (int q = 0; q < 4 * NM; ++q) mbar_init(x_bar + q, 64);
         mbar_init(mma_final, 1);
         fence_barrier_init();
     }
@@ -141,7 +139,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     if (warp == C::PRODUCER_WARP) {
         // compact the selected-block row: valid entries in order, bad ones recorded
         const int32_t* row = p.idx + ((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i) * p.topk;
-        int cnt = 0;
+        int cnt = 0, diag = -1;
         for (int t0 = 0; t0 < p.topk; t0 += 32) {
             const int t = t0 + lane;
             const int32_t j = t < p.topk ? row[t] : -1;
@@ -150,9 +148,16 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
             const int pos = cnt + __popc(m & ((1u << lane) - 1u));
             if (ok && pos < C::MAX_LIST) list[pos] = j;
+            // the diagonal block needs the per-token causal mask; its list position is found here
+            // once, so the softmax warps need no shared-memory read per key group
+            const uint32_t md = __ballot_sync(0xFFFFFFFFu, p.causal && ok && j == i && pos < C::MAX_LIST);
+            if (diag < 0 && md != 0u) diag = __shfl_sync(0xFFFFFFFFu, pos, __ffs(md) - 1);
             cnt += __popc(m);
         }
-        if (lane == 0) *s_nsel = cnt < C::MAX_LIST ? cnt : C::MAX_LIST;
+        if (lane == 0) {
+            *s_nsel = cnt < C::MAX_LIST ? cnt : C::MAX_LIST;
+            *s_diag = diag;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -160,6 +165,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     const uint32_t tm = *tmem_slot;
     const int nsel = *s_nsel;
     const int ngroups = (nsel + C::GB - 1) / C::GB;
+    const int diag_pos = *s_diag;
 
     int issued_last = -1;  // producer lanes: last group whose copies they started
     bool issued_any_mma = false;
@@ -204,7 +210,12 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         __syncwarp();
     } else if (warp == C::MMA_WARP) {
         if (lane == 0 && ngroups > 0) {
-            const uint32_t q_addr = smem_u32(Qs), k_addr = smem_u32(Ks), v_addr = smem_u32(Vs);
+            // Operand descriptors are formed once; every tile the MMAs read lies at a fixed offset
+            // from these bases. The start-address field holds address / 16 in 14 bits, and shared
+            // memory ends below 2^18 bytes, so adding offset / 16 never carries out of the field.
+            const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), C::SUB, 1024);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
             tc_fence_after();
@@ -216,13 +227,12 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                 const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
                 const uint32_t idesc_qk = idesc_bf16_f32(128, ncols, 0, 0);
                 const uint32_t d_tmem = tm + C::S_COL + h * 128;
+                const uint64_t a0 = dq0 + static_cast<uint32_t>((h * C::DS * C::SUB) >> 4);
+                const uint64_t b0 = dk0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t koff = (ks % 4) * 32;
-                    const uint64_t a = smem_desc_sw128(q_addr + (h * C::DS + ks / 4) * C::SUB + koff, 16, 1024);
-                    const uint64_t bd =
-                        smem_desc_sw128(k_addr + st * C::KG_BYTES + (ks / 4) * C::SUB + koff, 16, 1024);
-                    mma_bf16_ss(d_tmem, a, bd, idesc_qk, ks > 0 ? 1u : 0u);
+                    const uint32_t off = static_cast<uint32_t>(((ks / 4) * C::SUB + (ks % 4) * 32) >> 4);
+                    mma_bf16_ss(d_tmem, a0 + off, b0 + off, idesc_qk, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full + h);
                 issued_any_mma = true;
@@ -233,13 +243,17 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                 const int st = g % C::NST;
                 if (!mbar_wait(p_full + h, g & 1, p.status, detail_base | 0x14u)) return false;
                 tc_fence_after();
-                const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
+                const int nks = min(C::GB, nsel - g * C::GB) * BLK / 16;
                 const uint32_t d_tmem = tm + C::O_COL + h * D;
                 const uint32_t a_tmem = tm + C::S_COL + h * 128;
-                for (int ks = 0; ks < ncols / 16; ++ks) {
-                    const uint64_t bd = smem_desc_sw128(v_addr + st * C::KG_BYTES + ks * 16 * 128, C::SUB, 1024);
-                    const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
-                    mma_bf16_ts(d_tmem, a_tmem + acol, bd, idesc_pv, (g > 0 || ks > 0) ? 1u : 0u);
+                const uint64_t b0 = dv0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    if (ks < nks) {
+                        const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
+                        mma_bf16_ts(d_tmem, a_tmem + acol, b0 + static_cast<uint32_t>((ks * 16 * 128) >> 4), idesc_pv,
+                                    (g > 0 || ks > 0) ? 1u : 0u);
+                    }
                 }
                 mma_commit(pv_done + h);
                 return true;
@@ -277,20 +291,25 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         const int hh = R / BLK, t = R % BLK;
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const uint32_t s_tmem = tm + lane_base + C::S_COL + h * 128 + ch * 64;
-        // Row statistics meet through shared memory: this warp writes its value, both warps
-        // of the row quadrant arrive on x_bar, and each reads the other's value. The slots
-        // alternate with the exchange count, so a slot is rewritten only after the partner
-        // has passed the next exchange (and so has read it).
-        uint64_t* xb = x_bar + h * 4 + qd;
-        uint32_t n_xch = 0;
-        auto exchange = [&](float mine_v, float& other) -> bool {
-            float* slot = xch + (((n_xch & 1) * 2 + ch) * NM + h) * 128 + r;
-            *slot = mine_v;
-            mbar_arrive(xb);
-            const bool w = mbar_wait(xb, n_xch & 1, p.status, detail_base | 0x24u);
-            other = *(xch + (((n_xch & 1) * 2 + (ch ^ 1)) * NM + h) * 128 + r);
-            ++n_xch;
-            return w;
+        // Row statistics of the two warps of a row quadrant meet in TMEM: each warp writes its
+        // value into the last column of its own half of S (already read into registers), the
+        // pair meets at a named barrier, and each reads the partner's column. Shared memory is
+        // kept off this path: the tensor cores' operand reads keep it busy, and a shared access
+        // there waits hundreds of cycles. The barrier has no time limit, so the loop below never
+        // leaves early: after a failed wait a warp records the error, skips the remaining waits
+        // and keeps meeting its partner, once per key group and once in the epilogue.
+        const uint32_t xbar_id = 1u + static_cast<uint32_t>(h * 4 + qd);
+        const uint32_t slot_mine = s_tmem + 63;
+        const uint32_t slot_other = tm + lane_base + C::S_COL + h * 128 + (ch ^ 1) * 64 + 63;
+        auto exchange = [&](float mine_v) -> float {
+            tmem_st1(slot_mine, __float_as_uint(mine_v));
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar_sync(xbar_id, 64);
+            tc_fence_after();
+            const uint32_t o = tmem_ld1(slot_other);
+            tmem_wait_ld();
+            return __uint_as_float(o);
         };
         const float cs = p.scale_log2;
         const uint64_t cs2 = f2_pack(cs, cs);
@@ -300,26 +319,31 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             const int nb = min(C::GB, nsel - g * C::GB);
             const int ncols = nb * BLK;
             const int mine = max(0, min(64, ncols - ch * 64));  // columns of this half that hold keys
-            ok = mbar_wait(s_full + h, g & 1, p.status, detail_base | 0x20u);
-            if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full + h, g & 1, p.status, detail_base | 0x20u));
             tc_fence_after();
-            int diag_lo = 128;  // first column of the diagonal block, 128 if none
-            if (p.causal) {
-                for (int u = 0; u < nb; ++u)
-                    if (list[g * C::GB + u] == i) diag_lo = u * BLK;
-            }
+            // first column of the diagonal block, 128 if this group does not hold it
+            const int diag_lo = (diag_pos >= 0 && diag_pos / C::GB == g) ? (diag_pos % C::GB) * BLK : 128;
             const bool any_mask = ncols < 128 || diag_lo < 128;  // uniform across the CTA
             uint32_t pk[32];                                     // this half's P, bf16 pairs
             uint64_t sum2[2] = {0ull, 0ull};
+            float s_last = 0.f;  // raw score of this half's last column, whose TMEM cell the exchange reuses
             // exp2 of one 32-column chunk against the reference max; returns the chunk's max x.
-            // TRACK and MASKED are compile-time, so the unrolled pair loop has no branches and
-            // the compiler can interleave the sixteen independent pair chains.
-            auto chunk_exp = [&](int c, float m_ref, auto track_c, auto masked_c) -> float {
+            // TRACK, MASKED and PATCH are compile-time, so the unrolled pair loop has no branches
+            // and the compiler can interleave the sixteen independent pair chains. PATCH puts the
+            // saved last score back after an exchange has overwritten its cell.
+            auto chunk_exp = [&](int c, float m_ref, auto track_c, auto masked_c, auto patch_c) -> float {
                 constexpr bool TRACK = decltype(track_c)::value;
                 constexpr bool MASKED = decltype(masked_c)::value;
+                constexpr bool PATCH = decltype(patch_c)::value;
                 float sv[32];
                 tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
                 tmem_wait_ld();
+                if (c == 1) {
+                    if (PATCH)
+                        sv[31] = s_last;
+                    else
+                        s_last = sv[31];
+                }
                 if (MASKED) {
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
@@ -343,25 +367,60 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                 }
                 return xm;
             };
-            // fast path: probabilities against the running max, valid while no score of the
-            // row (in either half) exceeds it by more than the rescale threshold
-            bool redo = g == 0;
-            if (!redo) {
+            // exponentials of this half against m_ref, after the exchange (saved last score restored)
+            auto exps_patched = [&](float m_ref) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    if (c * 32 < mine) {
+                        if (any_mask)
+                            chunk_exp(c, m_ref, std::false_type{}, std::true_type{}, std::true_type{});
+                        else
+                            chunk_exp(c, m_ref, std::false_type{}, std::false_type{}, std::true_type{});
+                    }
+            };
+            float alpha = 1.0f, m_new = m_used;
+            if (g > 0) {
+                // fast path: probabilities against the running max m, kept while no score of the
+                // row (in either half) exceeds m by more than the rescale threshold
                 float xmax = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
                     if (c * 32 < mine)
-                        xmax = fmaxf(xmax, any_mask ? chunk_exp(c, m_used, std::true_type{}, std::true_type{})
-                                                    : chunk_exp(c, m_used, std::true_type{}, std::false_type{}));
-                float other;
-                ok = exchange(xmax, other);
-                if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-                xmax = fmaxf(xmax, other);
-                redo = __any_sync(0xFFFFFFFFu, xmax > kRescaleThreshold);
-            }
-            float alpha = 1.0f, m_new = m_used;
-            if (redo) {
-                // slow path (first group, or the max grew): the true row max, then the exponentials again
+                        xmax = fmaxf(xmax, any_mask ? chunk_exp(c, m_used, std::true_type{}, std::true_type{},
+                                                                std::false_type{})
+                                                    : chunk_exp(c, m_used, std::true_type{}, std::false_type{},
+                                                                std::false_type{}));
+                const float xall = fmaxf(xmax, exchange(xmax));  // row max of s*c - m over both halves
+                if (__any_sync(0xFFFFFFFFu, xall > kRescaleThreshold)) {
+                    // the row max grew past the threshold: m moves up to it, O is rescaled, and the
+                    // exponentials are redone from S
+                    const bool resc = xall > kRescaleThreshold;
+                    m_new = resc ? m_used + xall : m_used;
+                    alpha = resc ? fast_exp2(-xall) : 1.0f;
+                    if (ok && __any_sync(0xFFFFFFFFu, resc)) {
+                        // O holds P.V of every earlier group (its completion preceded this S); this
+                        // warp rescales its half of the columns
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x21u));
+                        if (ok) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int c = 0; c < D / 32; ++c) {
+                                uint32_t o[16];
+                                const uint32_t addr = tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 16;
+                                tmem_ld16(addr, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                                tmem_st16(addr, o);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) sum2[k] = 0ull;
+                    exps_patched(m_new);
+                }
+            } else {
+                // first group: the true row max, then the exponentials
                 float mq[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) mq[q] = -INFINITY;
@@ -371,6 +430,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                         float sv[32];
                         tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
                         tmem_wait_ld();
+                        if (c == 1) s_last = sv[31];
                         if (any_mask) {
 #pragma unroll
                             for (int k = 0; k < 32; ++k) {
@@ -383,41 +443,10 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                             mq[q] = fmax3(mq[q], sv[q], fmaxf(sv[8 + q], fmaxf(sv[16 + q], sv[24 + q])));
                     }
                 }
-                float mxs = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7]))) * cs;
-                float other;
-                ok = exchange(mxs, other);
-                if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-                mxs = fmaxf(mxs, other);
-                const bool resc = g > 0 && mxs > m_used + kRescaleThreshold;
-                m_new = (g == 0 || resc) ? mxs : m_used;
-                alpha = resc ? fast_exp2(m_used - m_new) : 1.0f;
-                if (g > 0 && __any_sync(0xFFFFFFFFu, resc)) {
-                    // O holds P.V of every earlier group (its completion preceded this S); this warp
-                    // rescales its half of the columns
-                    ok = mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x21u);
-                    if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[16];
-                        const uint32_t addr = tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 16;
-                        tmem_ld16(addr, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                        tmem_st16(addr, o);
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 2; ++k) sum2[k] = 0ull;
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    if (c * 32 < mine) {
-                        if (any_mask)
-                            chunk_exp(c, m_new, std::false_type{}, std::true_type{});
-                        else
-                            chunk_exp(c, m_new, std::false_type{}, std::false_type{});
-                    }
+                const float mxs =
+                    fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7]))) * cs;
+                m_new = fmaxf(mxs, exchange(mxs));
+                exps_patched(m_new);
             }
             // P overwrites this half's S columns, already read: 64 scores -> 32 columns
 #pragma unroll
@@ -432,45 +461,39 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             mbar_arrive(p_full + h);
         }
         // ---------------------------------------------------------------- epilogue
+        if (ok && ngroups > 0)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(pv_done + h, (ngroups - 1) & 1, p.status, detail_base | 0x22u));
+        const float l_sum = l_part + exchange(l_part);
         if (ok) {
             const int head = head0 + hh;
             const int64_t orow = (static_cast<int64_t>(b) * p.Hq + head) * p.N + static_cast<int64_t>(i) * BLK + t;
-            if (ngroups > 0) {
-                ok = mbar_wait(pv_done + h, (ngroups - 1) & 1, p.status, detail_base | 0x22u);
-                ok = __all_sync(0xFFFFFFFFu, ok);
-            }
-            float l_other = 0.f;
-            if (ok) ok = __all_sync(0xFFFFFFFFu, exchange(l_part, l_other));
-            const float l_sum = l_part + l_other;
-            if (ok) {
-                tc_fence_after();
-                const float inv = ngroups > 0 ? 1.0f / l_sum : 0.f;
-                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D + ch * (D / 2));
+            tc_fence_after();
+            const float inv = ngroups > 0 ? 1.0f / l_sum : 0.f;
+            uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D + ch * (D / 2));
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t o[32];
-                    if (ngroups > 0) {
-                        tmem_ld32(tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 32, o);
-                        tmem_wait_ld();
-                    } else {
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t o[32];
+                if (ngroups > 0) {
+                    tmem_ld32(tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 32, o);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = 0u;
-                    }
-                    if (valid) {
+                    for (int k = 0; k < 32; ++k) o[k] = 0u;
+                }
+                if (valid) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-                            dst[c * 4 + k] = v;
-                        }
+                    for (int k = 0; k < 4; ++k) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+                        dst[c * 4 + k] = v;
                     }
                 }
-                if (valid && ch == 0 && p.lse != nullptr)
-                    p.lse[orow] = ngroups > 0 ? (m_used + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             }
+            if (valid && ch == 0 && p.lse != nullptr)
+                p.lse[orow] = ngroups > 0 ? (m_used + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
         }
     }
 

@@ -231,3 +231,34 @@ def test_repeated_calls_are_deterministic(cuda_device):
     o2, l2, i2 = pisa.forward(shape, q, k, v, ws, idx=True)
     pisa.raise_on_device_error(ws)
     assert (i1 == i2).all() and (o1 == o2).all() and (l1 == l2).all()
+
+
+@pytest.mark.parametrize("causal", [0, 1])
+def test_growing_logits_rescale_running_max(causal, cuda_device):
+    """Key blocks scaled by factors that jump from block to block, with every block selected: the
+    row maximum grows past the lazy-rescale threshold at many key groups, sometimes in one
+    64-key half of a group and sometimes in both, so the running max, O and the row sums are
+    rescaled mid-row. The result must still be dense softmax attention."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    B, Hq, Hkv, nb, D, blk = 1, 8, 2, 24, 128, 64
+    N = nb * blk
+    gen = torch.Generator().manual_seed(41)
+    scale = torch.empty(nb).uniform_(0.3, 1.0, generator=gen) * torch.linspace(0.5, 4.0, nb)
+    scale[torch.randperm(nb, generator=gen)[:4]] *= 2.5
+    q = torch.randn((B, Hq, N, D), generator=gen)
+    k = torch.randn((B, Hkv, N, D), generator=gen) * scale.repeat_interleave(blk)[None, None, :, None]
+    v = torch.randn((B, Hkv, N, D), generator=gen)
+    q, k, v = (x.to(torch.bfloat16).to(cuda_device) for x in (q, k, v))
+    shape = pisa.Shape(B, Hq, Hkv, N, N, D, blk, 4, nb, causal=causal)
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws)
+    Q, K, V = (gu.host_f32(x) for x in (q, k, v))
+    o, lse = gu.host_f32(o), gu.host_f32(lse)
+    g = Hq // Hkv
+    sc = 1.0 / math.sqrt(D)
+    for h in range(Hq):
+        d_o, d_l = oracle.dense_attention(Q[0, h], np.arange(N), K[0, h // g], V[0, h // g], bool(causal), sc)
+        gu.assert_output_close(o[0, h], d_o, lse[0, h], d_l, f"causal={causal} h{h}")
