@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     const int head0 = p.per_qhead ? hs : kvh * p.g + chunk * p.gh;
     const uint32_t detail_base = kKernAttnPrefill << 8;
 
-    if (tid == 0) {
+    if (warp == C::PRODUCER_WARP && lane == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(k_full + s, 1);
@@ -134,6 +134,17 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         }
         mbar_init(mma_final, 1);
         fence_barrier_init();
+        // Q does not depend on the selection: its copy starts before the block row is read
+        prefetch_tmap(&tmQ);
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.gh * BLK * D * 2));
+        for (int hh = 0; hh < p.gh; ++hh) {
+            const int r0 = hh * BLK;
+            const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
+                                              static_cast<int64_t>(i) * BLK);
+#pragma unroll
+            for (int s = 0; s < C::DS; ++s)
+                tma_load_2d(Qs + ((r0 / 128) * C::DS + s) * C::SUB + (r0 % 128) * 128, &tmQ, s * 64, qrow, q_full);
+        }
     }
     if (warp == C::MMA_WARP) tmem_alloc(tmem_slot, C::TMEM_COLS);
     if (warp == C::PRODUCER_WARP) {
@@ -178,19 +189,6 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
             uint64_t* full = is_k ? k_full : v_full;
             uint64_t* empty = is_k ? k_empty : v_empty;
             prefetch_tmap(tmap);
-            if (is_k) {
-                prefetch_tmap(&tmQ);
-                mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.gh * BLK * D * 2));
-                for (int hh = 0; hh < p.gh; ++hh) {
-                    const int r0 = hh * BLK;
-                    const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
-                                                      static_cast<int64_t>(i) * BLK);
-#pragma unroll
-                    for (int s = 0; s < C::DS; ++s)
-                        tma_load_2d(Qs + ((r0 / 128) * C::DS + s) * C::SUB + (r0 % 128) * 128, &tmQ, s * 64, qrow,
-                                    q_full);
-                }
-            }
             for (int g = 0; g < ngroups; ++g) {
                 const int st = g % C::NST, use = g / C::NST;
                 if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
@@ -481,14 +479,15 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                     for (int k = 0; k < 32; ++k) o[k] = 0u;
                 }
                 if (valid) {
+                    // whole 32-byte sectors: each thread writes its row's columns 16 at a time
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-                        dst[c * 4 + k] = v;
+                    for (int k = 0; k < 2; ++k) {
+                        uint32_t v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            v[e] = pack_bf16x2(__uint_as_float(o[16 * k + 2 * e]) * inv,
+                                               __uint_as_float(o[16 * k + 2 * e + 1]) * inv);
+                        st_global_v8(dst + c * 4 + 2 * k, v);
                     }
                 }
             }
@@ -499,7 +498,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
 
     // ---------------------------------------------------------------- teardown
     __syncthreads();
-    if (warp == C::PRODUCER_WARP && lane < 2 && issued_last >= 0) {
+    if (warp == C::PRODUCER_WARP && lane < 2) {
         // every TMA load this CTA issued has landed before shared memory is released
         uint64_t* full = lane == 0 ? k_full : v_full;
         for (int g = max(0, issued_last - C::NST + 1); g <= issued_last; ++g)
