@@ -165,10 +165,11 @@ def _oracle_planes(w):
 def oracle_sample(w, budget_s: float = 15.0) -> dict:
     """Time the CPU oracle on a bounded sample of the workload; extrapolate to tokens/s.
 
-    Sample: the pyramid of one KV head (1/8 of the keys), the query summaries and
-    pyramid descent of up to 64 query blocks of that KV head, and the attention
-    of up to 8 query blocks (all 4 query heads each), stopping early when the
-    time budget is spent. Whole-problem time = per-unit times x unit counts.
+    Sample: the pyramid of one KV head (1/8 of the keys) and its query heads'
+    summaries, then the pyramid descent and the attention (all query heads of the
+    group) of seeded query blocks of that KV head, taken in a random order until
+    the time budget is spent (a third of it for the descent, the rest for the
+    attention). Whole-problem time = per-unit times x unit counts.
     """
     import oracle
     k, v, q_heads = _oracle_planes(w)
@@ -178,22 +179,22 @@ def oracle_sample(w, budget_s: float = 15.0) -> dict:
     t_pool = time.perf_counter() - t0          # one KV head's keys + its group's queries
     nqb = w.seq_q // w.block
     rng = np.random.Generator(np.random.PCG64(0))
-    blocks = sorted(set(rng.choice(nqb, size=min(64, nqb), replace=False).tolist()) | {nqb - 1})
+    order = [nqb - 1] + [int(x) for x in rng.permutation(nqb - 1)]
     sel = {}
     t0 = time.perf_counter()
-    for i in blocks:
+    for i in order:
         sel[i] = oracle.select_blocks(qbar[i], levels, w.factor, w.topk, i if w.causal else nqb - 1)["idx"]
         if time.perf_counter() - t0 > budget_s / 3:
             break
     t_sel = (time.perf_counter() - t0) / len(sel)
     t0 = time.perf_counter()
     n_att = 0
-    for i in list(sel)[:8]:
+    for i in sel:
         rows = np.arange(i * w.block, (i + 1) * w.block)
         for hh in range(w.group):
             oracle.attend(q_heads[hh, rows], rows, k, v, sel[i], w.block, bool(w.causal), 1 / np.sqrt(w.head_dim))
         n_att += 1
-        if time.perf_counter() - t0 > budget_s / 2:
+        if time.perf_counter() - t0 > budget_s * 2 / 3:
             break
     t_att = (time.perf_counter() - t0) / n_att
     units = w.batch * w.heads_kv
@@ -205,8 +206,8 @@ def oracle_sample(w, budget_s: float = 15.0) -> dict:
     except Exception:
         cores = os.cpu_count()
     return {"value": tokens / total, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
-            "sample": (f"pyramid+summaries of 1/{units} of the keys ({t_pool:.2f}s), descent of {len(sel)} query "
-                       f"blocks ({t_sel * 1e3:.1f} ms each), attention of {n_att} query blocks x {w.group} heads "
+            "sample": (f"pyramid+summaries of 1/{units} of the keys ({t_pool:.2f}s), descent of {len(sel)} random "
+                       f"query blocks ({t_sel * 1e3:.1f} ms each), attention of {n_att} of them x {w.group} heads "
                        f"({t_att * 1e3:.1f} ms each); extrapolated to {units} KV heads x {nqb} query blocks"),
             "seconds": round(t_pool + t_sel * len(sel) + t_att * n_att, 1),
             "estimated_full_seconds": round(total, 1)}
