@@ -33,7 +33,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 class PisaShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads_q", "heads_kv", "seq_q", "seq_kv", "head_dim",
                                                "block", "factor", "topk", "causal", "select_per_qhead")] + \
-               [("scale", ctypes.c_float)]
+               [("scale", ctypes.c_float), ("forced_blocks", ctypes.c_int32)]
+
+FORCE_SINK, FORCE_LOCAL = 1, 2   # pisa_shape.forced_blocks bits
 
 
 class PisaError(RuntimeError):
@@ -85,11 +87,12 @@ class Shape:
     causal: int = 0
     select_per_qhead: int = 0
     scale: float = 0.0
+    forced_blocks: int = 0   # FORCE_SINK | FORCE_LOCAL
 
     def c(self) -> PisaShape:
         return PisaShape(self.batch, self.heads_q, self.heads_kv, self.seq_q, self.seq_kv, self.head_dim,
                          self.block, self.factor, self.topk, int(self.causal), int(self.select_per_qhead),
-                         float(self.scale))
+                         float(self.scale), int(self.forced_blocks))
 
     @property
     def decode(self) -> bool:

@@ -21,7 +21,8 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     memset(p, 0, sizeof(*p));
     if (s->batch < 1 || s->heads_q < 1 || s->heads_kv < 1 || s->seq_q < 1 || s->seq_kv < 1 || s->head_dim < 1 ||
         s->block < 1 || s->factor < 2 || s->topk < 1 || (s->causal != 0 && s->causal != 1) ||
-        (s->select_per_qhead != 0 && s->select_per_qhead != 1) || !(s->scale == s->scale))
+        (s->select_per_qhead != 0 && s->select_per_qhead != 1) || !(s->scale == s->scale) ||
+        (s->forced_blocks & ~(PISA_FORCE_SINK | PISA_FORCE_LOCAL)) != 0)
         return PISA_ERR_INVALID_ARG;
     if (s->heads_q % s->heads_kv != 0) return PISA_ERR_INVALID_ARG;
     if (s->seq_kv % s->block != 0) return PISA_ERR_INVALID_ARG;
@@ -47,6 +48,7 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->decode = s->seq_q == 1 ? 1 : 0;
     p->causal = p->decode ? 0 : s->causal;
     p->per_qhead = s->select_per_qhead;
+    p->forced = s->forced_blocks;
     p->scale = s->scale > 0.f ? s->scale : 1.0f / sqrtf(static_cast<float>(s->head_dim));
     p->n0 = s->seq_kv / s->block;
 
@@ -185,6 +187,7 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
     sp.topk = pl.topk;
     sp.causal = pl.causal;
     sp.decode = pl.decode;
+    sp.forced = pl.forced;
     sp.L = pl.L;
     sp.total_nodes = pl.total_nodes;
     int64_t w = 1;

@@ -261,6 +261,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int a_mn, in
            | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
 }
 
+// ---------------------------------------------------------------- selection variants
+
+// Forced blocks of one query block (PISA_FORCE_* mask): key block 0 for the sink, `local`
+// (the query's own block) for the local block, ascending, at most `cap` of them, the sink
+// first. Returns how many; unused outputs are -1.
+__device__ __forceinline__ int forced_blocks(int32_t mask, int32_t local, int32_t cap, int32_t& f0, int32_t& f1) {
+    int n = 0;
+    f0 = -1;
+    f1 = -1;
+    if (mask & PISA_FORCE_SINK) {
+        f0 = 0;
+        n = 1;
+    }
+    if ((mask & PISA_FORCE_LOCAL) && !(n == 1 && local == 0)) {
+        if (n == 0) {
+            f0 = local;
+            n = 1;
+        } else if (cap >= 2) {
+            f1 = local;
+            n = 2;
+        }
+    }
+    return n < cap ? n : cap;
+}
+
 // ---------------------------------------------------------------- small math
 
 __device__ __forceinline__ float fast_exp2(float x) {

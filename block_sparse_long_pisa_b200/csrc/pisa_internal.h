@@ -39,6 +39,7 @@ enum : uint32_t {
 // Derived sizes of one problem (host side).
 struct Plan {
     int32_t B, Hq, Hkv, g, Nq, N, D, blk, f, topk, causal, per_qhead, decode;
+    int32_t forced;      // PISA_FORCE_* bit mask
     float scale;
     int32_t n0;          // key blocks per sequence
     int32_t L;           // pyramid levels
@@ -91,6 +92,7 @@ struct SelectParams {
     float* margin;              // optional fp32 [B, Hsel, nqb]
     uint32_t* status;
     int32_t Hsel, Hkv, gsel_div, nqb, D, n0, factor, topk, causal, decode, L, total_nodes;
+    int32_t forced;             // PISA_FORCE_* bit mask
     int32_t lsize[PISA_MAX_LEVELS];
     int32_t loff[PISA_MAX_LEVELS];
     int32_t budget[PISA_MAX_LEVELS];

@@ -19,6 +19,8 @@
 //    scores, lower index. The kept nodes' eligible children become the next
 //    candidates; holes (ineligible children) carry key 0 and sort last.
 // 5. The kept level-0 blocks are written in ascending order, padded with -1.
+//    Forced blocks (sink, local) are left out of the level-0 candidates, which
+//    then keep K minus their count, and join the output before the final sort.
 #include <cuda_bf16.h>
 
 #include "pisa_device.cuh"
@@ -148,6 +150,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     }
     int nkeep;
     int32_t* out_ids = cand;  // reused for the final ascending sort
+    int32_t f0, f1;
+    const int nf = forced_blocks(p.forced, p.decode ? p.n0 - 1 : i, p.budget[0], f0, f1);
     if (l0 < 0) {
         nkeep = last + 1;  // every eligible block fits the budget
         const int n = next_pow2(nkeep);
@@ -155,8 +159,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
         __syncthreads();
     } else {
         int ncand = static_cast<int>(last / p.width[l0] + 1);
-        for (int t = tid; t < ncand; t += kSelThreads) cand[t] = t;
-        if (tid == 0) s_nvalid = ncand;
+        // at level 0 the forced blocks (all eligible) are not candidates
+        for (int t = tid; t < ncand; t += kSelThreads) cand[t] = (l0 == 0 && (t == f0 || t == f1)) ? -1 : t;
+        if (tid == 0) s_nvalid = l0 == 0 ? ncand - nf : ncand;
         __syncthreads();
         nkeep = 0;
         for (int l = l0; l >= 0; --l) {
@@ -202,9 +207,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             __syncthreads();
             const int nvalid = s_nvalid;
             bitonic_desc(keys, n);
-            const int k_l = p.budget[l];
+            const int k_l = l == 0 ? p.budget[0] - nf : p.budget[l];
             nkeep = min(k_l, nvalid);
-            if (tid == 0 && nvalid > k_l) {
+            if (tid == 0 && nvalid > k_l && k_l > 0) {
                 const float a = order_bits_inv(static_cast<uint32_t>(keys[k_l - 1] >> 32));
                 const float c = order_bits_inv(static_cast<uint32_t>(keys[k_l] >> 32));
                 const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
@@ -221,7 +226,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
                 for (int t = tid; t < slots; t += kSelThreads) {
                     const int32_t c = key_node(keys[t / p.factor]);
                     const int64_t ch = static_cast<int64_t>(c) * p.factor + (t % p.factor);
-                    const bool ok = ch <= last_below && ch < n_below;
+                    const bool ok = ch <= last_below && ch < n_below && (l > 1 || (ch != f0 && ch != f1));
                     cand[t] = ok ? static_cast<int32_t>(ch) : -1;
                     mine += ok;
                 }
@@ -229,9 +234,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
                 ncand = slots;
                 __syncthreads();
             } else {
-                const int nn = next_pow2(nkeep);
+                const int nn = next_pow2(nkeep + nf);
                 __syncthreads();
-                for (int t = tid; t < nn; t += kSelThreads) out_ids[t] = t < nkeep ? key_node(keys[t]) : 0x7FFFFFFF;
+                for (int t = tid; t < nn; t += kSelThreads)
+                    out_ids[t] = t < nkeep ? key_node(keys[t]) : t < nkeep + nf ? (t == nkeep ? f0 : f1) : 0x7FFFFFFF;
+                nkeep += nf;
                 __syncthreads();
             }
         }

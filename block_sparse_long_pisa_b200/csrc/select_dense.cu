@@ -206,6 +206,9 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
 
     const float* srow = p.scores + row * p.total_nodes;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    // forced blocks (sink, local): not candidates at level 0, added to the output at the end
+    int32_t f0, f1;
+    const int nf = forced_blocks(p.forced, i, p.budget[0], f0, f1);
     float margin = __int_as_float(0x7F800000);
     int32_t node[J];
     {
@@ -214,6 +217,11 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
         for (int j = 0; j < J; ++j) node[j] = 32 * j + lane < cnt0 ? 32 * j + lane : -1;
     }
     for (int l = l0;; --l) {
+        if (l == 0 && nf > 0) {
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+                if (node[j] == f0 || node[j] == f1) node[j] = -1;
+        }
         const int64_t c_part = last / p.width[l];
         const bool has_part = min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
         const float ps = has_part ? pscore[l] : 0.f;
@@ -227,10 +235,10 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
             nv += v;
         }
         const int nvalid = __reduce_add_sync(FULL, nv);
-        const int K = p.budget[l];
+        const int K = l == 0 ? p.budget[0] - nf : p.budget[l];
         // kept: hi > t_hi, or hi == t_hi and ~node >= t_lo; invalid candidates have hi == 0
         uint32_t t_hi = 1u, t_lo = 0u;
-        if (nvalid > K) {
+        if (K > 0 && nvalid > K) {
             // MSB-first bisection for the K-th largest score bits; it stops as soon as a
             // tested threshold keeps exactly K candidates (the cut then falls between
             // two distinct scores), which takes about log2(candidates) + a few steps
@@ -290,14 +298,29 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
         int nkeep = 0;
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-            const bool keep = hi[j] > t_hi || (hi[j] == t_hi && ~static_cast<uint32_t>(node[j]) >= t_lo);
+            // (K == 0: every slot of the level is taken by forced blocks, no candidate is kept)
+            const bool keep = K > 0 && (hi[j] > t_hi || (hi[j] == t_hi && ~static_cast<uint32_t>(node[j]) >= t_lo));
             const uint32_t bal = __ballot_sync(FULL, keep);
             if (keep) kl[nkeep + __popc(bal & lt_mask)] = node[j];
             nkeep += __popc(bal);
         }
         __syncwarp();
         if (l == 0) {
-            for (int t = lane; t < p.topk; t += 32) dst[t] = t < nkeep ? kl[t] : -1;
+            // merge the forced blocks into the ascending list of kept blocks (none of them is kept)
+            int below0 = 0, below1 = 0;
+            for (int t = lane; t < nkeep; t += 32) {
+                const int32_t v = kl[t];
+                dst[t + (nf >= 1 && f0 < v) + (nf >= 2 && f1 < v)] = v;
+                below0 += v < f0;
+                below1 += v < f1;
+            }
+            below0 = __reduce_add_sync(FULL, below0);
+            below1 = __reduce_add_sync(FULL, below1);
+            if (lane == 0) {
+                if (nf >= 1) dst[below0] = f0;
+                if (nf >= 2) dst[below1 + 1] = f1;
+            }
+            for (int t = nkeep + nf + lane; t < p.topk; t += 32) dst[t] = -1;
             if (p.margin != nullptr && lane == 0) p.margin[row] = margin;
             return;
         }

@@ -63,13 +63,26 @@ typedef struct CUstream_st *pisa_stream_t;
  *   select_per_qhead         : 0 = one selection per (batch, KV head, query block) from the
  *                              mean over the g query heads (default); 1 = one selection per
  *                              query head.
- *   scale                    : softmax scale; <= 0 selects 1/sqrt(head_dim). */
+ *   scale                    : softmax scale; <= 0 selects 1/sqrt(head_dim).
+ *   forced_blocks            : selection variant (PISA page, section "Ce que PISA change
+ *                              concretement": top-K variants per domain; Pulsar Attention page,
+ *                              section "Phase 1": a fixed attention-sink prefix). Bit mask of
+ *                              PISA_FORCE_SINK (key block 0) and PISA_FORCE_LOCAL (the query's own
+ *                              block: block i for prefill, the last block for decode). A forced
+ *                              block is always selected; the descent fills the other
+ *                              K - (forced blocks) slots at level 0 from the remaining candidates
+ *                              (coarser levels keep their budgets). At most K forced blocks are
+ *                              kept, the sink first. 0 = plain top-K (default). */
 typedef struct {
     int32_t batch, heads_q, heads_kv, seq_q, seq_kv, head_dim;
     int32_t block, factor, topk, causal;
     int32_t select_per_qhead;
     float scale;
+    int32_t forced_blocks;
 } pisa_shape;
+
+#define PISA_FORCE_SINK 1
+#define PISA_FORCE_LOCAL 2
 
 typedef enum {
     PISA_OK = 0,

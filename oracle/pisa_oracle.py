@@ -135,8 +135,19 @@ def rank_key(score_value: float, node: int) -> tuple[float, int]:
     return (-float(score_value), node)
 
 
+def forced_set(forced: int, local: int, topk: int) -> list[int]:
+    """Blocks a selection variant always keeps (R16): key block 0 (attention sink, bit 1) and the
+    query's own block `local` (bit 2), without repeats, at most K of them, the sink first."""
+    out: list[int] = []
+    if forced & 1:
+        out.append(0)
+    if forced & 2 and local not in out:
+        out.append(local)
+    return out[:topk]
+
+
 def select_blocks(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk: int,
-                  last: int, budgets: list[int] | None = None) -> dict:
+                  last: int, budgets: list[int] | None = None, forced: list[int] | None = None) -> dict:
     """Descend the pyramid for one query summary and keep the top-K key blocks.
 
     Start with every eligible node of the top level; at each level score the
@@ -145,6 +156,10 @@ def select_blocks(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk:
     default). Returns the kept level-0 blocks sorted ascending (R12), the
     smallest relative margin s_(K) - s_(K+1) met at a pruning level (R10), and
     the number of candidates scored (work bound, O(N log N)).
+
+    `forced` (R16) lists level-0 blocks that are always kept: they are taken out
+    of the level-0 candidates, whose budget drops by their number, and added to
+    the result. Coarser levels are unchanged.
     """
     n_levels = len(levels)
     n0 = levels[0].shape[0]
@@ -155,12 +170,17 @@ def select_blocks(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk:
     margin = math.inf
     n_scored = 0
     kept: list[int] = []
+    forced = [] if forced is None else list(forced)
     for l in range(top, -1, -1):
+        if l == 0 and forced:
+            cands = [c for c in cands if c not in forced]
         scores = [score(qbar, node_value(levels, factor, l, c, last)) for c in cands]
         n_scored += len(cands)
         order = sorted(range(len(cands)), key=lambda t: rank_key(scores[t], cands[t]))
-        k_l = budgets[l]
-        if len(cands) > k_l:
+        k_l = budgets[l] - (len(forced) if l == 0 else 0)
+        if k_l == 0:
+            kept = []
+        elif len(cands) > k_l:
             s_k, s_k1 = float(scores[order[k_l - 1]]), float(scores[order[k_l]])
             rel = (s_k - s_k1) / max(abs(s_k), abs(s_k1), 1e-30)
             margin = min(margin, rel)
@@ -171,7 +191,7 @@ def select_blocks(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk:
             n_below = levels[l - 1].shape[0]
             cands = sorted(ch for c in kept for ch in children(n_below, factor, c)
                            if node_span(n0, factor, l - 1, ch)[0] <= last)
-    return {"idx": sorted(kept), "margin": margin, "n_scored": n_scored}
+    return {"idx": sorted(kept + forced), "margin": margin, "n_scored": n_scored}
 
 
 # ----------------------------------------------------------------------------- attention
@@ -254,7 +274,8 @@ def selection_heads(heads_q: int, heads_kv: int, per_qhead: bool, hs: int) -> tu
 
 def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int, factor: int, topk: int,
             causal: bool, scale: float | None = None, per_qhead: bool = False,
-            budgets: list[int] | None = None, idx_override: np.ndarray | None = None) -> dict:
+            budgets: list[int] | None = None, idx_override: np.ndarray | None = None,
+            forced: int = 0) -> dict:
     """Pyramid -> query summaries -> descent top-K -> sparse attention, for whole tensors.
 
     Q [B, Hq, Nq, D] (Nq = N for prefill, 1 for decode at position N-1), K, V
@@ -280,7 +301,8 @@ def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int, factor: int
             qbar = query_summary(Q[b, heads], 1 if decode else block)
             for i in range(nqb):
                 last = n0 - 1 if (decode or not causal) else i
-                r = select_blocks(qbar[i], pyr[b][kvh], factor, topk, last, budgets)
+                fset = forced_set(forced, n0 - 1 if decode else i, topk)
+                r = select_blocks(qbar[i], pyr[b][kvh], factor, topk, last, budgets, fset)
                 idx[b, hs, i, :len(r["idx"])] = r["idx"]
                 margin[b, hs, i] = r["margin"]
                 n_scored[b, hs, i] = r["n_scored"]

@@ -292,6 +292,77 @@ def check_work_bound(o, seed=19, N=4096, block=16, factor=4, topk=8, D=16):
     assert r["n_scored"] < nb
 
 
+# ----------------------------------------------------------------------------- R16 forced blocks
+
+def brute_topk_excluding(qbar, k_plane, block, topk, last, excluded):
+    """Exhaustive top-K over eligible level-0 blocks not in `excluded` (fp64, lower index on ties)."""
+    nb = k_plane.shape[0] // block
+    means = k_plane.astype(np.float64).reshape(nb, block, -1).mean(axis=1)
+    s = means[:last + 1] @ qbar.astype(np.float64)
+    pool = [j for j in range(last + 1) if j not in excluded]
+    order = sorted(pool, key=lambda j: (-s[j], j))
+    if len(pool) <= topk:
+        return sorted(order), math.inf
+    if topk == 0:
+        return [], math.inf
+    a, b = s[order[topk - 1]], s[order[topk]]
+    return sorted(order[:topk]), (a - b) / max(abs(a), abs(b), 1e-30)
+
+
+def check_forced_full_budgets(o, forced, seed=21, causal=True, N=1024, block=16, factor=4, topk=8, D=16):
+    """With K_l = n_l at the coarse levels, a selection with forced blocks F equals F plus the
+    exhaustive top-(K - |F|) of the other eligible blocks."""
+    q, k, v = rand_qkv(seed, 1, 2, 1, N, N, D)
+    levels = o.build_pyramid(k[0, 0], block, factor)
+    budgets = [topk] + [lev.shape[0] for lev in levels[1:]]
+    qbar = o.query_summary(q[0], block)
+    nb = N // block
+    checked = 0
+    for i in range(nb):
+        last = i if causal else nb - 1
+        fset = []
+        if forced & 1:
+            fset.append(0)
+        if forced & 2 and i not in fset:
+            fset.append(i)
+        fset = fset[:topk]
+        rest, margin = brute_topk_excluding(qbar[i], k[0, 0], block, topk - len(fset), last, fset)
+        if margin < 1e-4:
+            continue
+        got = o.select_blocks(qbar[i], levels, factor, topk, last, budgets, o.forced_set(forced, i, topk))["idx"]
+        assert got == sorted(rest + fset), (i, got, sorted(rest + fset))
+        checked += 1
+    assert checked > nb // 2
+
+
+def check_forced_cardinality(o, seed=22, topk=3, N=512, block=16, factor=4):
+    """Every row keeps min(K, eligible) distinct sorted blocks and holds its forced blocks."""
+    q, k, v = rand_qkv(seed, 1, 2, 1, N, N, 16)
+    nb = N // block
+    for forced in (1, 2, 3):
+        res = o.forward(q, k, v, block, factor, topk, True, forced=forced)
+        for i in range(nb):
+            row = res["idx"][0, 0, i]
+            valid = row[row >= 0]
+            assert len(valid) == min(topk, i + 1), (forced, i, row)
+            assert np.all(np.diff(valid) > 0) and valid.max() <= i
+            if forced & 1:
+                assert 0 in valid
+            if forced & 2:
+                assert i in valid
+
+
+def check_forced_budget_edges(o, seed=23, N=256, block=16, factor=4):
+    """K = 1 with sink and local: the sink alone; K = 2: the sink and the query's own block."""
+    q, k, v = rand_qkv(seed, 1, 1, 1, N, N, 16)
+    nb = N // block
+    r1 = o.forward(q, k, v, block, factor, 1, True, forced=3)["idx"][0, 0]
+    assert np.all(r1[:, 0] == 0)
+    r2 = o.forward(q, k, v, block, factor, 2, True, forced=3)["idx"][0, 0]
+    for i in range(nb):
+        assert r2[i].tolist() == ([0, -1] if i == 0 else [0, i]), (i, r2[i])
+
+
 ALL_PINS = {
     "pyramid_means": check_pyramid_means,
     "query_summary": check_query_summary,
@@ -310,4 +381,9 @@ ALL_PINS = {
     "causal_partial_node": check_causal_partial_node,
     "causal_invariance": check_causal_invariance,
     "work_bound": check_work_bound,
+    "forced_sink_full_budgets": lambda o: check_forced_full_budgets(o, 1),
+    "forced_local_full_budgets_noncausal": lambda o: check_forced_full_budgets(o, 2, causal=False),
+    "forced_both_full_budgets": lambda o: check_forced_full_budgets(o, 3),
+    "forced_cardinality": check_forced_cardinality,
+    "forced_budget_edges": check_forced_budget_edges,
 }

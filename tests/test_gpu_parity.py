@@ -38,12 +38,12 @@ PER_QHEAD = {
 }
 
 
-def _run(w, cuda_device, per_qhead=False, topk=None):
+def _run(w, cuda_device, per_qhead=False, topk=None, forced=0):
     import torch
     import block_sparse_long_pisa_b200 as pisa
     if topk is not None:
         w = w.replace(topk=topk)
-    shape = pisa.Shape.of(w, select_per_qhead=int(per_qhead))
+    shape = pisa.Shape.of(w, select_per_qhead=int(per_qhead), forced_blocks=forced)
     q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
     ws = pisa.new_workspace(shape, cuda_device)
     o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
@@ -52,7 +52,7 @@ def _run(w, cuda_device, per_qhead=False, topk=None):
     pisa.raise_on_device_error(ws, w.name)
     assert pisa.last_launch_count() >= 1
     Q, K, V = (gu.host_f32(x) for x in (q, k, v))
-    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_qhead)
+    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_qhead, forced=forced)
     return shape, (Q, K, V), ref, gu.host_f32(o), gu.host_f32(lse), idx.cpu().numpy(), gu.host_f32(pyr)
 
 
@@ -262,3 +262,44 @@ def test_growing_logits_rescale_running_max(causal, cuda_device):
     for h in range(Hq):
         d_o, d_l = oracle.dense_attention(Q[0, h], np.arange(N), K[0, h // g], V[0, h // g], bool(causal), sc)
         gu.assert_output_close(o[0, h], d_o, lse[0, h], d_l, f"causal={causal} h{h}")
+
+
+FORCED_CASES = [("tiny", 3), ("gqa4-causal-ragged", 1), ("gqa4-causal-ragged", 2), ("gqa4-causal-ragged", 3),
+                ("gqa4-causal-short", 3), ("decode-gqa4", 3), ("decode-d64-b128", 2), ("perq-gqa4-causal", 3),
+                ("mha-d128-b128-f8-causal", 1)]
+
+
+@pytest.mark.parametrize("name,forced", FORCED_CASES)
+def test_forced_blocks_match_oracle(name, forced, cuda_device):
+    """Selection variants (attention sink, local block, both) on both selection paths (dense
+    prefill scoring, per-query-block descent for short prefill and decode) and per-query-head."""
+    per_q = name in PER_QHEAD
+    w = PER_QHEAD[name] if per_q else SMALL[name]
+    shape, (Q, K, V), ref, o, lse, idx, _ = _run(w, cuda_device, per_qhead=per_q, forced=forced)
+    bad, near = gu.selection_report(idx, ref["idx"], ref["margin"])
+    assert bad == 0, f"{bad} selections differ outside near-ties ({near} near-ties)"
+    nqb = 1 if w.decode else w.seq_q // w.block
+    n0 = w.n_blocks
+    for i in range(nqb):
+        local = n0 - 1 if w.decode else i
+        rows = idx[:, :, i]
+        if forced & 1:
+            assert np.all((rows == 0).any(axis=-1))
+        if forced & 2:
+            assert np.all((rows == local).any(axis=-1))
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_q, idx_override=idx)
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"], name)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_forced_blocks_fill_the_budget(topk, cuda_device):
+    """K no larger than the forced blocks: K = 1 keeps the sink alone, K = 2 the sink and the
+    query's own block, on both selection paths."""
+    for name in ("gqa4-causal-ragged", "gqa4-causal-short"):
+        w = SMALL[name]
+        _, _, ref, _, _, idx, _ = _run(w, cuda_device, topk=topk, forced=3)
+        assert np.array_equal(idx, ref["idx"]), name
+        nqb = w.seq_q // w.block
+        for i in range(nqb):
+            expect = [0] if topk == 1 else ([0, -1] if i == 0 else [0, i])
+            assert np.all(idx[:, :, i] == np.array(expect)), (name, i)

@@ -69,6 +69,27 @@ def _score_dropped_component(qbar, node):
     return F32(np.dot(qbar[1:].astype(F32), node[1:].astype(F32)))
 
 
+def _forced_not_truncated(forced, local, topk):
+    out = [0] if forced & 1 else []
+    if forced & 2 and local not in out:
+        out.append(local)
+    return out
+
+
+def _forced_repeats_sink(forced, local, topk):
+    out = [0] if forced & 1 else []
+    if forced & 2:
+        out.append(local)
+    return out[:topk]
+
+
+def _forced_local_is_previous_block(forced, local, topk):
+    out = [0] if forced & 1 else []
+    if forced & 2 and max(local - 1, 0) not in out:
+        out.append(max(local - 1, 0))
+    return out[:topk]
+
+
 def _one_level_too_many(n0, factor):
     sizes = [n0]
     while sizes[-1] >= factor:
@@ -89,6 +110,9 @@ MUTATIONS = {
     "merge weights with the wrong sign": ("merge_partials", _merge_wrong_sign),
     "score drops one component": ("score", _score_dropped_component),
     "pyramid builds one level too many": ("level_sizes", _one_level_too_many),
+    "forced blocks exceed K": ("forced_set", _forced_not_truncated),
+    "sink repeated as the local block": ("forced_set", _forced_repeats_sink),
+    "local block off by one": ("forced_set", _forced_local_is_previous_block),
 }
 
 
