@@ -64,9 +64,10 @@ typedef struct CUstream_st *pisa_stream_t;
  *                              mean over the g query heads (default); 1 = one selection per
  *                              query head.
  *   scale                    : softmax scale; <= 0 selects 1/sqrt(head_dim).
- *   forced_blocks            : selection variant (PISA page, section "Ce que PISA change
- *                              concretement": top-K variants per domain; Pulsar Attention page,
- *                              section "Phase 1": a fixed attention-sink prefix). Bit mask of
+ *   forced_blocks            : selection variant (PISA page, section "Ce que cela change pour
+ *                              vous": top-K variants per domain; Pulsar Attention page, section
+ *                              "Phase 1 : Encodage statistique du contexte": a fixed
+ *                              attention-sink prefix). Bit mask of
  *                              PISA_FORCE_SINK (key block 0) and PISA_FORCE_LOCAL (the query's own
  *                              block: block i for prefill, the last block for decode). A forced
  *                              block is always selected; the descent fills the other
