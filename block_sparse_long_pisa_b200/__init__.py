@@ -33,7 +33,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 class PisaShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads_q", "heads_kv", "seq_q", "seq_kv", "head_dim",
                                                "block", "factor", "topk", "causal", "select_per_qhead")] + \
-               [("scale", ctypes.c_float), ("forced_blocks", ctypes.c_int32)]
+               [("scale", ctypes.c_float), ("forced_blocks", ctypes.c_int32), ("kv_capacity", ctypes.c_int32)]
 
 FORCE_SINK, FORCE_LOCAL = 1, 2   # pisa_shape.forced_blocks bits
 
@@ -56,6 +56,7 @@ _sig = {
     "pisa_pyramid_size": (ctypes.c_int, [_SP, _szp]),
     "pisa_workspace_size": (ctypes.c_int, [_SP, _szp]),
     "pisa_build_pyramid": (ctypes.c_int, [_SP, _vp, _vp, _vp]),
+    "pisa_append_pyramid": (ctypes.c_int, [_SP, _vp, _vp, ctypes.c_int32, _vp]),
     "pisa_select_blocks": (ctypes.c_int, [_SP, _vp, _vp, _i32p, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "pisa_sparse_attention": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "pisa_forward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -88,11 +89,12 @@ class Shape:
     select_per_qhead: int = 0
     scale: float = 0.0
     forced_blocks: int = 0   # FORCE_SINK | FORCE_LOCAL
+    kv_capacity: int = 0     # decode over a growing cache: K/V rows per plane (0 = seq_kv)
 
     def c(self) -> PisaShape:
         return PisaShape(self.batch, self.heads_q, self.heads_kv, self.seq_q, self.seq_kv, self.head_dim,
                          self.block, self.factor, self.topk, int(self.causal), int(self.select_per_qhead),
-                         float(self.scale), int(self.forced_blocks))
+                         float(self.scale), int(self.forced_blocks), int(self.kv_capacity))
 
     @property
     def decode(self) -> bool:
@@ -101,6 +103,11 @@ class Shape:
     @property
     def n_blocks(self) -> int:
         return self.seq_kv // self.block
+
+    @property
+    def kv_rows(self) -> int:
+        """Rows of one K/V plane: the capacity of a growing cache, else seq_kv."""
+        return self.kv_capacity or self.seq_kv
 
     @property
     def hsel(self) -> int:
@@ -191,12 +198,21 @@ def new_workspace(shape: Shape, device) -> "object":
 def build_pyramid(shape: Shape, K, pyramid=None, stream=None):
     torch = _torch()
     D = shape.head_dim
-    _need(K, torch.bfloat16, (shape.batch, shape.heads_kv, shape.seq_kv, D), "K")
+    _need(K, torch.bfloat16, (shape.batch, shape.heads_kv, shape.kv_rows, D), "K")
     sizes, _ = level_layout(shape)
     if pyramid is None:
         pyramid = torch.empty((shape.batch, shape.heads_kv, sum(sizes), D), dtype=torch.float32, device=K.device)
     _check(_lib.pisa_build_pyramid(ctypes.byref(shape.c()), _ptr(K), _ptr(pyramid), _stream(stream)),
            "pisa_build_pyramid")
+    return pyramid
+
+
+def append_pyramid(shape: Shape, K, pyramid, seq_kv_old: int, stream=None):
+    """Brings `pyramid` (the pyramid of the cache at length seq_kv_old) up to shape.seq_kv."""
+    torch = _torch()
+    _need(K, torch.bfloat16, (shape.batch, shape.heads_kv, shape.kv_rows, shape.head_dim), "K")
+    _check(_lib.pisa_append_pyramid(ctypes.byref(shape.c()), _ptr(K), _ptr(pyramid), int(seq_kv_old), _stream(stream)),
+           "pisa_append_pyramid")
     return pyramid
 
 
@@ -232,8 +248,8 @@ def forward(shape: Shape, Q, K, V, ws, O=None, lse=True, idx=None, stream=None):
     torch = _torch()
     B, Hq, Nq, D = shape.batch, shape.heads_q, shape.seq_q, shape.head_dim
     _need(Q, torch.bfloat16, (B, Hq, Nq, D), "Q")
-    _need(K, torch.bfloat16, (B, shape.heads_kv, shape.seq_kv, D), "K")
-    _need(V, torch.bfloat16, (B, shape.heads_kv, shape.seq_kv, D), "V")
+    _need(K, torch.bfloat16, (B, shape.heads_kv, shape.kv_rows, D), "K")
+    _need(V, torch.bfloat16, (B, shape.heads_kv, shape.kv_rows, D), "V")
     if O is None:
         O = torch.empty_like(Q)
     L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=Q.device) if lse is True else lse

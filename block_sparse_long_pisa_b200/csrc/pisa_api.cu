@@ -27,11 +27,14 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     if (s->heads_q % s->heads_kv != 0) return PISA_ERR_INVALID_ARG;
     if (s->seq_kv % s->block != 0) return PISA_ERR_INVALID_ARG;
     if (s->seq_q != s->seq_kv && s->seq_q != 1) return PISA_ERR_INVALID_ARG;
+    const int32_t cap = s->kv_capacity == 0 ? s->seq_kv : s->kv_capacity;
+    if (cap < s->seq_kv || cap % s->block != 0) return PISA_ERR_INVALID_ARG;
+    if (s->seq_q != 1 && cap != s->seq_kv) return PISA_ERR_INVALID_ARG;  // capacity: decode only
     if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
     if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
     // every row index must fit the 32-bit TMA coordinate and grid limits
     const int64_t qrows = static_cast<int64_t>(s->batch) * s->heads_q * s->seq_q;
-    const int64_t krows = static_cast<int64_t>(s->batch) * s->heads_kv * s->seq_kv;
+    const int64_t krows = static_cast<int64_t>(s->batch) * s->heads_kv * cap;
     if (qrows >= (int64_t(1) << 31) || krows >= (int64_t(1) << 31)) return PISA_ERR_UNSUPPORTED;
     if (s->batch > 65535) return PISA_ERR_UNSUPPORTED;
 
@@ -40,7 +43,7 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->Hkv = s->heads_kv;
     p->g = s->heads_q / s->heads_kv;
     p->Nq = s->seq_q;
-    p->N = s->seq_kv;
+    p->N = cap;
     p->D = s->head_dim;
     p->blk = s->block;
     p->f = s->factor;
@@ -51,8 +54,9 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->forced = s->forced_blocks;
     p->scale = s->scale > 0.f ? s->scale : 1.0f / sqrtf(static_cast<float>(s->head_dim));
     p->n0 = s->seq_kv / s->block;
+    p->n0_cap = cap / s->block;
 
-    int n = p->n0, L = 0, off = 0;
+    int n = p->n0_cap, L = 0, off = 0;
     while (true) {
         if (L >= PISA_MAX_LEVELS) return PISA_ERR_UNSUPPORTED;
         p->lsize[L] = n;
@@ -114,7 +118,13 @@ static int heads_per_cta(const Plan& pl) {
     return best;
 }
 
-static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cudaStream_t st) {
+// Pyramid nodes over level-0 blocks [b_lo, b_hi) (and over no block when the range is empty at
+// a level), bottom-up: level-0 means of those blocks, then at every coarser level the nodes
+// whose span meets the range. A full build is the range [0, n0_cap): blocks past n0 (spare
+// capacity) come out as zeros.
+static pisa_status pyramid_range(const Plan& pl, const void* K, float* pyr, int32_t b_lo, int32_t b_hi,
+                                 cudaStream_t st) {
+    if (b_hi <= b_lo) return PISA_OK;
     MeanParams m{};
     m.src = static_cast<const __nv_bfloat16*>(K);
     m.dst = pyr;
@@ -122,7 +132,9 @@ static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cuda
     m.Nsrc = pl.N;
     m.D = pl.D;
     m.Hout = pl.Hkv;
-    m.rows_out = pl.n0;
+    m.row0 = b_lo;
+    m.rows_out = b_hi - b_lo;
+    m.rows_valid = pl.n0;
     m.dst_plane_rows = pl.total_nodes;
     m.rows_per_group = pl.blk;
     m.planes_per_group = 1;
@@ -131,6 +143,9 @@ static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cuda
     ++g_launches;
     int64_t width = 1;
     for (int l = 1; l < pl.L; ++l) {
+        const int64_t wl = width * pl.f;
+        const int32_t c_lo = static_cast<int32_t>(b_lo / wl);
+        const int32_t c_hi = static_cast<int32_t>(min(static_cast<int64_t>(pl.lsize[l]), (b_hi - 1) / wl + 1));
         LevelParams lp{};
         lp.pyr = pyr;
         lp.planes = pl.B * pl.Hkv;
@@ -138,16 +153,21 @@ static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cuda
         lp.off_below = pl.loff[l - 1];
         lp.off_cur = pl.loff[l];
         lp.n_below = pl.lsize[l - 1];
-        lp.n_cur = pl.lsize[l];
+        lp.c0 = c_lo;
+        lp.n_cur = c_hi - c_lo;
         lp.n0 = pl.n0;
         lp.factor = pl.f;
         lp.D = pl.D;
         lp.width_below = width;
         if (!launch_pyramid_level(lp, st)) return PISA_ERR_CUDA;
         ++g_launches;
-        width *= pl.f;
+        width = wl;
     }
     return PISA_OK;
+}
+
+static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cudaStream_t st) {
+    return pyramid_range(pl, K, pyr, 0, pl.n0_cap, st);
 }
 
 static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cudaStream_t st) {
@@ -159,6 +179,8 @@ static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cud
     m.D = pl.D;
     m.Hout = pl.Hsel;
     m.rows_out = pl.nqb;
+    m.row0 = 0;
+    m.rows_valid = pl.nqb;
     m.dst_plane_rows = pl.nqb;
     m.rows_per_group = pl.decode ? 1 : pl.blk;
     m.planes_per_group = pl.gsel;
@@ -182,7 +204,8 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
     sp.gsel_div = pl.per_qhead ? pl.g : 1;
     sp.nqb = pl.nqb;
     sp.D = pl.D;
-    sp.n0 = pl.n0;
+    sp.n0 = pl.n0_cap;
+    sp.n0_valid = pl.n0;
     sp.factor = pl.f;
     sp.topk = pl.topk;
     sp.causal = pl.causal;
@@ -306,6 +329,17 @@ pisa_status pisa_build_pyramid(const pisa_shape* shape, const void* K, float* py
     if (s != PISA_OK) return s;
     if (K == nullptr || pyramid == nullptr || !aligned16(K) || !aligned16(pyramid)) return PISA_ERR_INVALID_ARG;
     return build_pyramid(pl, K, pyramid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pisa_status pisa_append_pyramid(const pisa_shape* shape, const void* K, float* pyramid, int32_t seq_kv_old,
+                                pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    const pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (K == nullptr || pyramid == nullptr || !aligned16(K) || !aligned16(pyramid)) return PISA_ERR_INVALID_ARG;
+    if (seq_kv_old < 0 || seq_kv_old > shape->seq_kv || seq_kv_old % pl.blk != 0) return PISA_ERR_INVALID_ARG;
+    return pyramid_range(pl, K, pyramid, seq_kv_old / pl.blk, pl.n0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 static pisa_status check_budget(const Plan& pl, const int32_t* level_budget) {

@@ -41,7 +41,8 @@ struct Plan {
     int32_t B, Hq, Hkv, g, Nq, N, D, blk, f, topk, causal, per_qhead, decode;
     int32_t forced;      // PISA_FORCE_* bit mask
     float scale;
-    int32_t n0;          // key blocks per sequence
+    int32_t n0;          // key blocks that hold keys (seq_kv / block)
+    int32_t n0_cap;      // key blocks of the capacity (kv_capacity / block); the pyramid layout's n_0
     int32_t L;           // pyramid levels
     int32_t lsize[PISA_MAX_LEVELS];
     int32_t loff[PISA_MAX_LEVELS];
@@ -68,7 +69,9 @@ struct MeanParams {
     float* dst;                 // fp32 rows
     int32_t Hsrc, Nsrc, D;
     int32_t Hout;               // output planes per batch
-    int32_t rows_out;           // output rows per plane (n0 or nqb)
+    int32_t rows_out;           // output rows per plane computed by this launch
+    int32_t row0;               // first output row (rows row0 .. row0 + rows_out - 1)
+    int32_t rows_valid;         // rows at or past this index have no data: written as zeros
     int32_t dst_plane_rows;     // row stride between output planes
     int32_t rows_per_group;     // source rows averaged per output row (block, or 1)
     int32_t planes_per_group;   // consecutive source heads averaged (g or 1)
@@ -80,8 +83,9 @@ struct LevelParams {
     int32_t planes;             // batch * heads_kv
     int32_t plane_rows;         // total_nodes
     int32_t off_below, off_cur; // row offsets of the two levels inside a plane
-    int32_t n_below, n_cur;
-    int32_t n0, factor, D;
+    int32_t n_below, n_cur;     // n_cur: nodes computed by this launch, from node c0 on
+    int32_t c0;
+    int32_t n0, factor, D;      // n0: level-0 blocks that hold keys (the weights count only these)
     int64_t width_below;        // level-0 blocks under one node of the level below (f^(l-1))
 };
 
@@ -91,7 +95,9 @@ struct SelectParams {
     int32_t* idx;               // int32 [B, Hsel, nqb, topk]
     float* margin;              // optional fp32 [B, Hsel, nqb]
     uint32_t* status;
-    int32_t Hsel, Hkv, gsel_div, nqb, D, n0, factor, topk, causal, decode, L, total_nodes;
+    int32_t Hsel, Hkv, gsel_div, nqb, D, factor, topk, causal, decode, L, total_nodes;
+    int32_t n0;                 // level-0 blocks of the pyramid layout (node spans)
+    int32_t n0_valid;           // level-0 blocks that hold keys (decode: the last one is the query's)
     int32_t forced;             // PISA_FORCE_* bit mask
     int32_t lsize[PISA_MAX_LEVELS];
     int32_t loff[PISA_MAX_LEVELS];

@@ -7,8 +7,13 @@
 // once, so the kernel is bound by HBM bandwidth.
 //
 // pyramid_level_kernel: one thread per (plane, node, 4 floats); a node of
-// level l is the mean of its children weighted by the level-0 blocks each
-// child covers (the last node of a level may have fewer than f children).
+// level l is the mean of its children weighted by the level-0 blocks holding
+// keys that each child covers (the last node of a level may have fewer than f
+// children; in a cache with spare capacity, nodes past the keys weigh 0, and a
+// node over no key at all is 0).
+//
+// Both kernels compute a contiguous range of rows or nodes, so that appending
+// blocks to a KV cache recomputes only what changed, with the same arithmetic.
 #include <cuda_bf16.h>
 
 #include "pisa_device.cuh"
@@ -40,7 +45,7 @@ __global__ void __launch_bounds__(256) block_mean_kernel(const MeanParams p) {
     const int lane = threadIdx.x & 31;
     const int64_t total = static_cast<int64_t>(p.batch) * p.Hout * p.rows_out;
     if (warp >= total) return;
-    const int i = static_cast<int>(warp % p.rows_out);
+    const int i = p.row0 + static_cast<int>(warp % p.rows_out);
     const int hs = static_cast<int>((warp / p.rows_out) % p.Hout);
     const int b = static_cast<int>(warp / (static_cast<int64_t>(p.rows_out) * p.Hout));
     const int chunk = lane % CH;
@@ -50,7 +55,7 @@ __global__ void __launch_bounds__(256) block_mean_kernel(const MeanParams p) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 
-    for (int pp = 0; pp < p.planes_per_group; ++pp) {
+    for (int pp = 0; pp < (i < p.rows_valid ? p.planes_per_group : 0); ++pp) {
         const int64_t head = static_cast<int64_t>(hs) * p.planes_per_group + pp;
         const __nv_bfloat16* base = p.src + ((static_cast<int64_t>(b) * p.Hsrc + head) * p.Nsrc +
                                              static_cast<int64_t>(i) * p.rows_per_group) * D + chunk * 8;
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(256) pyramid_level_kernel(const LevelParams p)
     const int64_t total = static_cast<int64_t>(p.planes) * p.n_cur * q4;
     if (t >= total) return;
     const int q = static_cast<int>(t % q4);
-    const int c = static_cast<int>((t / q4) % p.n_cur);
+    const int c = p.c0 + static_cast<int>((t / q4) % p.n_cur);
     const int64_t plane = t / (static_cast<int64_t>(q4) * p.n_cur);
     const float* below = p.pyr + (plane * p.plane_rows + p.off_below) * p.D + 4 * q;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -96,6 +101,7 @@ __global__ void __launch_bounds__(256) pyramid_level_kernel(const LevelParams p)
         if (ch >= p.n_below) break;
         const int64_t lo = ch * p.width_below;
         const int64_t hi = min((ch + 1) * p.width_below, static_cast<int64_t>(p.n0));
+        if (hi <= lo) break;  // this child and the ones after it hold no key
         const float w = static_cast<float>(hi - lo);
         const float4 v = *reinterpret_cast<const float4*>(below + ch * p.D);
         acc.x += w * v.x;
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(256) pyramid_level_kernel(const LevelParams p)
         acc.w += w * v.w;
         wsum += hi - lo;
     }
-    const float inv = 1.0f / static_cast<float>(wsum);
+    const float inv = wsum > 0 ? 1.0f / static_cast<float>(wsum) : 0.f;
     float* dst = p.pyr + (plane * p.plane_rows + p.off_cur + c) * p.D + 4 * q;
     *reinterpret_cast<float4*>(dst) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }

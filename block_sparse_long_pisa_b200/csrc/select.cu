@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     const int i = blockIdx.x, hs = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x;
     const int kvh = hs / p.gsel_div;
-    const int last = (p.causal && !p.decode) ? i : p.n0 - 1;
+    const int last = (p.causal && !p.decode) ? i : p.n0_valid - 1;
     const float* plane = p.pyr + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.total_nodes * D;
     const int64_t row = (static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i;
 
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     int nkeep;
     int32_t* out_ids = cand;  // reused for the final ascending sort
     int32_t f0, f1;
-    const int nf = forced_blocks(p.forced, p.decode ? p.n0 - 1 : i, p.budget[0], f0, f1);
+    const int nf = forced_blocks(p.forced, p.decode ? p.n0_valid - 1 : i, p.budget[0], f0, f1);
     if (l0 < 0) {
         nkeep = last + 1;  // every eligible block fits the budget
         const int n = next_pow2(nkeep);

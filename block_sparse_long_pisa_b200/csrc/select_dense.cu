@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kScThreads, 2) score_kernel(const SelectParams
     const int i0 = (tile / p.tiles_c[l]) * kScTile;
     const int c0 = (tile % p.tiles_c[l]) * kScTile;
     const int i_hi = min(i0 + kScTile, p.nqb) - 1;
-    const int64_t last_hi = p.causal ? i_hi : p.n0 - 1;
+    const int64_t last_hi = p.causal ? i_hi : p.n0_valid - 1;
     // the start level and the eligible range only grow with the query block
     if (start_level(p, last_hi) < l || c0 > last_hi / p.width[l]) return;
 
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
     const int hs = static_cast<int>((row / p.nqb) % p.Hsel);
     const int b = static_cast<int>(row / (static_cast<int64_t>(p.nqb) * p.Hsel));
     const int kvh = hs / p.gsel_div;
-    const int64_t last = p.causal ? i : p.n0 - 1;
+    const int64_t last = p.causal ? i : p.n0_valid - 1;
     int32_t* dst = p.idx + row * p.topk;
     const int l0 = start_level(p, last);
     if (l0 < 0) {  // every eligible block fits the budget

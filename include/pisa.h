@@ -73,13 +73,19 @@ typedef struct CUstream_st *pisa_stream_t;
  *                              block is always selected; the descent fills the other
  *                              K - (forced blocks) slots at level 0 from the remaining candidates
  *                              (coarser levels keep their budgets). At most K forced blocks are
- *                              kept, the sink first. 0 = plain top-K (default). */
+ *                              kept, the sink first. 0 = plain top-K (default).
+ *   kv_capacity              : decode over a growing KV cache: K and V are [B, Hkv, kv_capacity,
+ *                              D] of which the first seq_kv positions hold keys; the pyramid
+ *                              layout (levels, offsets, size) is that of kv_capacity, so it does
+ *                              not move as the cache grows (pisa_append_pyramid). A multiple of
+ *                              block, >= seq_kv. 0 means seq_kv. Prefill requires 0 or seq_kv. */
 typedef struct {
     int32_t batch, heads_q, heads_kv, seq_q, seq_kv, head_dim;
     int32_t block, factor, topk, causal;
     int32_t select_per_qhead;
     float scale;
     int32_t forced_blocks;
+    int32_t kv_capacity;
 } pisa_shape;
 
 #define PISA_FORCE_SINK 1
@@ -125,11 +131,30 @@ PISA_API pisa_status pisa_workspace_size(const pisa_shape *shape, size_t *bytes)
 /* Step 1, the key pyramid ("Le pooling comme premiere reduction"): level 0 is
  * the fp32 mean of every key block of `block` keys; a node of level l+1 is the
  * mean of its children weighted by the level-0 blocks each covers (so every
- * node is the mean of all keys under it).
- *   K        : bf16 [batch, heads_kv, seq_kv, head_dim], device.
+ * node is the mean of all keys under it). With spare capacity (kv_capacity >
+ * seq_kv) only the first seq_kv / block blocks hold keys: the weights count
+ * those alone, and a node over none of them is 0.
+ *   K        : bf16 [batch, heads_kv, kv_capacity (or seq_kv), head_dim], device.
  *   pyramid  : fp32 output, pisa_pyramid_size bytes, device. */
 PISA_API pisa_status pisa_build_pyramid(const pisa_shape *shape, const void *K, float *pyramid,
                                pisa_stream_t stream);
+
+/* Keeps a pyramid current as a KV cache grows, without rebuilding it (incremental pyramid
+ * maintenance for decode; PISA page, section "Le pooling comme premiere reduction": each level
+ * summarises the one below). `pyramid` must hold the pyramid of the cache at length
+ * `seq_kv_old` (from pisa_build_pyramid or an earlier append with the same kv_capacity; a
+ * zero-filled buffer is the pyramid of an empty cache). The call computes the level-0 means of
+ * the blocks completed since, [seq_kv_old / block, seq_kv / block), and every coarser node over
+ * them, with the arithmetic of pisa_build_pyramid: the result equals a build at seq_kv bit for
+ * bit. Work is O((new blocks) * block * D + L * f * D) per plane, not O(seq_kv * D).
+ *   shape      : the cache after the append (seq_kv = new length, kv_capacity as before).
+ *   K          : bf16 [B, Hkv, kv_capacity, D], device.
+ *   pyramid    : fp32, device, pisa_pyramid_size bytes, updated in place.
+ *   seq_kv_old : 0 <= seq_kv_old <= seq_kv, a multiple of block.
+ * Errors: PISA_ERR_INVALID_ARG for a bad shape, null or misaligned pointers or a bad
+ * seq_kv_old; PISA_ERR_CUDA if a launch fails. Asynchronous on `stream`. */
+PISA_API pisa_status pisa_append_pyramid(const pisa_shape *shape, const void *K, float *pyramid,
+                                         int32_t seq_kv_old, pisa_stream_t stream);
 
 /* Step 2, pyramid-guided top-K ("La selection top-K guidee par la pyramide").
  * For every query block: its summary q = mean of its queries (over the g query

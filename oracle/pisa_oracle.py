@@ -93,6 +93,39 @@ def build_pyramid(k_plane: np.ndarray, block: int, factor: int) -> list[np.ndarr
     return levels
 
 
+def build_pyramid_capacity(k_plane: np.ndarray, block: int, factor: int, kv_len: int) -> list[np.ndarray]:
+    """Key pyramid of a KV cache with spare capacity (R17): k_plane [capacity, D] of which the
+    first kv_len rows hold keys. The levels have the sizes of the whole capacity; every node is
+    the mean of the keys it covers among the first kv_len (weights count only those blocks), and
+    a node over none of them is 0. With kv_len = capacity this is ``build_pyramid``.
+    """
+    n0_cap = k_plane.shape[0] // block
+    nv = kv_len // block
+    d = k_plane.shape[1]
+    sizes = level_sizes(n0_cap, factor)
+    lev0 = np.zeros((n0_cap, d), dtype=F32)
+    if nv > 0:
+        lev0[:nv] = block_means(k_plane[:nv * block], block)
+    levels = [lev0]
+    for l in range(1, len(sizes)):
+        below = levels[l - 1]
+        cur = np.zeros((sizes[l], d), dtype=F32)
+        for c in range(sizes[l]):
+            acc = np.zeros(d, dtype=F32)
+            total = 0
+            for ch in children(sizes[l - 1], factor, c):
+                lo, hi = node_span(n0_cap, factor, l - 1, ch)
+                cnt = max(0, min(hi, nv - 1) - lo + 1)
+                if cnt == 0:
+                    continue
+                acc += F32(cnt) * below[ch]
+                total += cnt
+            if total > 0:
+                cur[c] = acc / F32(total)
+        levels.append(cur)
+    return levels
+
+
 # ----------------------------------------------------------------------------- query summary
 
 def query_summary(q_heads: np.ndarray, rows_per_block: int) -> np.ndarray:
@@ -275,23 +308,31 @@ def selection_heads(heads_q: int, heads_kv: int, per_qhead: bool, hs: int) -> tu
 def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int, factor: int, topk: int,
             causal: bool, scale: float | None = None, per_qhead: bool = False,
             budgets: list[int] | None = None, idx_override: np.ndarray | None = None,
-            forced: int = 0) -> dict:
+            forced: int = 0, kv_len: int | None = None) -> dict:
     """Pyramid -> query summaries -> descent top-K -> sparse attention, for whole tensors.
 
     Q [B, Hq, Nq, D] (Nq = N for prefill, 1 for decode at position N-1), K, V
     [B, Hkv, N, D], all bf16-exact fp32. Selection is shared by the g query heads
     of a KV head unless per_qhead. `idx_override` replaces the oracle's own
     selection in the attention step (used to check attention on given indices).
+    Decode over a cache with spare capacity (R17): K and V hold `kv_len` keys
+    followed by unused rows; the pyramid has the capacity's levels and the query
+    sits at position kv_len - 1.
     """
     B, Hq, Nq, D = Q.shape
-    Hkv, N = K.shape[1], K.shape[2]
+    Hkv, N_rows = K.shape[1], K.shape[2]
+    N = N_rows if kv_len is None else kv_len
     g = Hq // Hkv
     decode = Nq == 1
+    assert kv_len is None or decode, "spare KV capacity is a decode feature"
     sc = default_scale(D, scale)
     n0 = N // block
     hsel = Hq if per_qhead else Hkv
     nqb = 1 if decode else Nq // block
-    pyr = [[build_pyramid(K[b, h], block, factor) for h in range(Hkv)] for b in range(B)]
+    if kv_len is None:
+        pyr = [[build_pyramid(K[b, h], block, factor) for h in range(Hkv)] for b in range(B)]
+    else:
+        pyr = [[build_pyramid_capacity(K[b, h], block, factor, kv_len) for h in range(Hkv)] for b in range(B)]
     idx = np.full((B, hsel, nqb, topk), -1, dtype=np.int32)
     margin = np.full((B, hsel, nqb), np.inf, dtype=np.float64)
     n_scored = np.zeros((B, hsel, nqb), dtype=np.int64)

@@ -363,6 +363,47 @@ def check_forced_budget_edges(o, seed=23, N=256, block=16, factor=4):
         assert r2[i].tolist() == ([0, -1] if i == 0 else [0, i]), (i, r2[i])
 
 
+# ----------------------------------------------------------------------------- R17 spare KV capacity
+
+def check_capacity_pyramid_means(o, seed=24, n_cap=37, block=16, factor=4, D=12):
+    """Every node of a capacity pyramid is the fp64 mean of the keys it covers among the first
+    kv_len rows, and 0 when it covers none of them."""
+    rng = _rng(seed)
+    k = _bf16_exact(rng.standard_normal((n_cap * block, D)))
+    for nv in (0, 1, 5, 16, 21, n_cap):
+        levels = o.build_pyramid_capacity(k, block, factor, nv * block)
+        width = 1
+        for l, lev in enumerate(levels):
+            for c in range(lev.shape[0]):
+                lo, hi = c * width * block, min((c + 1) * width, nv) * block
+                expect = k[lo:hi].astype(np.float64).mean(axis=0) if hi > lo else np.zeros(D)
+                assert np.allclose(lev[c], expect, atol=1e-5, rtol=1e-5), (nv, l, c)
+            width *= factor
+
+
+def check_capacity_decode_equals_exact(o, seed=25, n_cap=64, nv=39, block=16, factor=4, topk=5, D=16):
+    """Decode on a cache with spare capacity selects what decode on the exact-length cache
+    selects (outside near-ties) and gives the same attention."""
+    q, k, v = rand_qkv(seed, 2, 4, 2, 1, n_cap * block, D)
+    kv_len = nv * block
+    cap = o.forward(q, k, v, block, factor, topk, False, kv_len=kv_len)
+    exact = o.forward(q, k[:, :, :kv_len], v[:, :, :kv_len], block, factor, topk, False)
+    same = np.all(cap["idx"] == exact["idx"], axis=-1)
+    near = (cap["margin"] < 1e-3) | (exact["margin"] < 1e-3)
+    assert np.all(same | near)
+    assert same.sum() >= same.size // 2
+    for b in range(2):
+        for h in range(4):
+            if same[b, h // 2, 0]:
+                assert np.allclose(cap["O"][b, h], exact["O"][b, h], atol=1e-6)
+    # the spare rows are never read: garbage there changes nothing
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, kv_len:] = 1e4
+    v2[:, :, kv_len:] = -1e4
+    cap2 = o.forward(q, k2, v2, block, factor, topk, False, kv_len=kv_len)
+    assert np.array_equal(cap2["idx"], cap["idx"]) and np.array_equal(cap2["O"], cap["O"])
+
+
 ALL_PINS = {
     "pyramid_means": check_pyramid_means,
     "query_summary": check_query_summary,
@@ -386,4 +427,6 @@ ALL_PINS = {
     "forced_both_full_budgets": lambda o: check_forced_full_budgets(o, 3),
     "forced_cardinality": check_forced_cardinality,
     "forced_budget_edges": check_forced_budget_edges,
+    "capacity_pyramid_means": check_capacity_pyramid_means,
+    "capacity_decode_equals_exact": check_capacity_decode_equals_exact,
 }

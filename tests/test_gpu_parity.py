@@ -303,3 +303,72 @@ def test_forced_blocks_fill_the_budget(topk, cuda_device):
         for i in range(nqb):
             expect = [0] if topk == 1 else ([0, -1] if i == 0 else [0, i])
             assert np.all(idx[:, :, i] == np.array(expect)), (name, i)
+
+
+def _capacity_cache(w, cap, cuda_device):
+    """K and V of a decode workload placed in a cache of `cap` rows; the spare rows hold NaN,
+    so any read past the keys would show in the results."""
+    import torch
+    k, v = (gu.to_device(w, t, cuda_device) for t in ("k", "v"))
+    out = []
+    for x in (k, v):
+        c = torch.full((w.batch, w.heads_kv, cap, w.head_dim), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+        c[:, :, :w.seq_kv] = x
+        out.append(c)
+    return out
+
+
+def test_capacity_pyramid_build_and_append(cuda_device):
+    """A cache with spare capacity: the pyramid built at one length matches the oracle; appending
+    blocks (one at a time and several at once) gives the pyramid a build at the new length gives,
+    bit for bit."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL["decode-gqa4"]                  # 45 blocks of 64 keys
+    cap = 64 * 64
+    kc, _ = _capacity_cache(w, cap, cuda_device)
+    kc = torch.nan_to_num(kc, nan=0.0)        # rows past a length are never averaged, but keep them finite
+    K = gu.host_f32(kc)
+
+    def shape_at(n):
+        return pisa.Shape(w.batch, w.heads_q, w.heads_kv, 1, n, w.head_dim, w.block, w.factor, w.topk,
+                          kv_capacity=cap)
+    lengths = [17 * 64, 18 * 64, 19 * 64, 30 * 64, 45 * 64]
+    pyr = pisa.build_pyramid(shape_at(lengths[0]), kc)
+    _, offs = pisa.level_layout(shape_at(lengths[0]))
+    for n_old, n_new in zip(lengths, lengths[1:]):
+        pisa.append_pyramid(shape_at(n_new), kc, pyr, n_old)
+        fresh = pisa.build_pyramid(shape_at(n_new), kc)
+        torch.cuda.synchronize()
+        assert torch.equal(pyr, fresh), (n_old, n_new)
+        got = gu.host_f32(pyr)
+        for b in range(w.batch):
+            for h in range(w.heads_kv):
+                ref = oracle.build_pyramid_capacity(K[b, h], w.block, w.factor, n_new)
+                gu.assert_pyramid_close(got[b, h], ref, offs)
+
+
+@pytest.mark.parametrize("forced", [0, 3])
+def test_decode_with_spare_capacity(forced, cuda_device):
+    """Decode over a partly filled cache (spare rows hold NaN) matches the oracle's decode at the
+    cache's current length."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL["decode-gqa4"]
+    cap = 80 * 64
+    kc, vc = _capacity_cache(w, cap, cuda_device)
+    q = gu.to_device(w, "q", cuda_device)
+    shape = pisa.Shape.of(w, kv_capacity=cap, forced_blocks=forced)
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, kc, vc, ws, idx=True)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws)
+    Q, K, V = gu.host_f32(q), gu.host_f32(kc), gu.host_f32(vc)
+    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, kv_len=w.seq_kv, forced=forced)
+    idx = idx.cpu().numpy()
+    bad, _ = gu.selection_report(idx, ref["idx"], ref["margin"])
+    assert bad == 0
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, kv_len=w.seq_kv, idx_override=idx)
+    o, lse = gu.host_f32(o), gu.host_f32(lse)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"], "spare capacity")

@@ -90,6 +90,10 @@ def _forced_local_is_previous_block(forced, local, topk):
     return out[:topk]
 
 
+def _capacity_counts_spare_blocks(k_plane, block, factor, kv_len):
+    return po.build_pyramid(k_plane, block, factor)
+
+
 def _one_level_too_many(n0, factor):
     sizes = [n0]
     while sizes[-1] >= factor:
@@ -113,6 +117,7 @@ MUTATIONS = {
     "forced blocks exceed K": ("forced_set", _forced_not_truncated),
     "sink repeated as the local block": ("forced_set", _forced_repeats_sink),
     "local block off by one": ("forced_set", _forced_local_is_previous_block),
+    "capacity pyramid averages the spare rows": ("build_pyramid_capacity", _capacity_counts_spare_blocks),
 }
 
 
