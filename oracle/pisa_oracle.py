@@ -291,6 +291,73 @@ def merge_partials(outs: list[np.ndarray], lses: list[np.ndarray]) -> tuple[np.n
     return o, lse
 
 
+# ----------------------------------------------------------------------------- backward
+
+def attend_backward(q_rows: np.ndarray, q_pos: np.ndarray, k_plane: np.ndarray, v_plane: np.ndarray,
+                    blocks: list[int], block: int, causal: bool, scale: float, d_out: np.ndarray
+                    ) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients of ``attend`` (fp64) through a fixed selection: the selection itself has no
+    gradient (it is a discrete choice), the softmax over the selected keys does.
+
+    With S = scale Q K_sel^T (masked), P = softmax(S) row by row and O = P V_sel:
+      dV_sel = P^T dO,  dP = dO V_sel^T,  dS = P * (dP - rowsum(dO * O)),
+      dQ = scale dS K_sel,  dK_sel = scale dS^T Q.
+    Returns dQ [R, D] and dK, dV over the whole plane [N, D] (zero outside the selected keys).
+    """
+    dq = np.zeros(q_rows.shape, dtype=np.float64)
+    dk = np.zeros(k_plane.shape, dtype=np.float64)
+    dv = np.zeros(v_plane.shape, dtype=np.float64)
+    if len(blocks) == 0:
+        return dq, dk, dv
+    key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
+    q = q_rows.astype(np.float64)
+    kx = k_plane[key_pos].astype(np.float64)
+    vx = v_plane[key_pos].astype(np.float64)
+    do = d_out.astype(np.float64)
+    s = scale * (q @ kx.T)
+    if causal:
+        s = np.where(key_pos[None, :] > q_pos[:, None], -np.inf, s)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p /= p.sum(axis=1, keepdims=True)
+    o = p @ vx
+    dvx = p.T @ do
+    dp = do @ vx.T
+    ds = p * (dp - (do * o).sum(axis=1, keepdims=True))
+    dq = scale * (ds @ kx)
+    np.add.at(dk, key_pos, scale * (ds.T @ q))
+    np.add.at(dv, key_pos, dvx)
+    return dq, dk, dv
+
+
+def backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.ndarray, idx: np.ndarray, block: int,
+             causal: bool, scale: float | None = None, per_qhead: bool = False) -> dict:
+    """dQ, dK, dV (fp64) of the sparse attention step for given selected blocks `idx`
+    [B, Hsel, nqb, K] (prefill): per query block and head, ``attend_backward``; a KV head's
+    dK and dV sum the contributions of all its query heads (GQA)."""
+    B, Hq, N, D = Q.shape
+    Hkv = K.shape[1]
+    g = Hq // Hkv
+    sc = default_scale(D, scale)
+    nqb = N // block
+    dQ = np.zeros(Q.shape, dtype=np.float64)
+    dK = np.zeros(K.shape, dtype=np.float64)
+    dV = np.zeros(V.shape, dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // g
+            hs = h if per_qhead else kvh
+            for i in range(nqb):
+                rows = np.arange(i * block, (i + 1) * block)
+                blocks = [int(j) for j in idx[b, hs, i] if j >= 0]
+                dq, dk, dv = attend_backward(Q[b, h, rows], rows, K[b, kvh], V[b, kvh], blocks, block, causal,
+                                             sc, dO[b, h, rows])
+                dQ[b, h, rows] = dq
+                dK[b, kvh] += dk
+                dV[b, kvh] += dv
+    return {"dQ": dQ, "dK": dK, "dV": dV}
+
+
 # ----------------------------------------------------------------------------- whole forward
 
 def default_scale(head_dim: int, scale: float | None) -> float:

@@ -404,6 +404,88 @@ def check_capacity_decode_equals_exact(o, seed=25, n_cap=64, nv=39, block=16, fa
     assert np.array_equal(cap2["idx"], cap["idx"]) and np.array_equal(cap2["O"], cap["O"])
 
 
+# ----------------------------------------------------------------------------- backward
+
+def _loss_sparse(o, Q, K, V, W, idx, block, causal, scale):
+    """sum(O * W) of the sparse attention step, from the fp64 dense softmax with a mask that
+    keeps each query block's selected keys (an independent route to the same forward)."""
+    B, Hq, N, D = Q.shape
+    g = Hq // K.shape[1]
+    total = 0.0
+    for b in range(B):
+        for h in range(Hq):
+            allowed = np.zeros((N, N), dtype=bool)
+            for i in range(N // block):
+                for j in idx[b, h // g, i]:
+                    if j >= 0:
+                        allowed[i * block:(i + 1) * block, j * block:(j + 1) * block] = True
+            out, _ = o.dense_attention(Q[b, h], np.arange(N), K[b, h // g], V[b, h // g], causal, scale, allowed)
+            total += float((out * W[b, h]).sum())
+    return total
+
+
+def check_backward_finite_differences(o, seed=26, causal=True, B=1, Hq=2, Hkv=1, nb=4, block=8, D=8, topk=2):
+    """dQ, dK, dV of the sparse step match central finite differences of sum(O * dO) taken
+    through the fp64 dense forward with the selection as a mask."""
+    rng = _rng(seed)
+    N = nb * block
+    Q, K, V = (rng.standard_normal((B, h, N, D)) for h in (Hq, Hkv, Hkv))
+    W = rng.standard_normal((B, Hq, N, D))
+    idx = np.full((B, Hkv, nb, topk), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(nb):
+                elig = i + 1 if causal else nb
+                sel = np.sort(rng.choice(elig, size=min(topk, elig), replace=False))
+                idx[b, h, i, :len(sel)] = sel
+    scale = 0.7
+    g = o.backward(Q, K, V, W, idx, block, causal, scale)
+    eps = 1e-6
+    for name, T in (("dQ", Q), ("dK", K), ("dV", V)):
+        for _ in range(12):
+            pos = tuple(int(rng.integers(0, n)) for n in T.shape)
+            old = T[pos]
+            T[pos] = old + eps
+            lp = _loss_sparse(o, Q, K, V, W, idx, block, causal, scale)
+            T[pos] = old - eps
+            lm = _loss_sparse(o, Q, K, V, W, idx, block, causal, scale)
+            T[pos] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - g[name][pos]) < 1e-6 + 1e-5 * abs(fd), (name, pos, fd, g[name][pos])
+
+
+def check_backward_constant_values(o, seed=27, N=64, block=16, D=8):
+    """When every key has the same value row, O does not depend on the scores: dQ = dK = 0,
+    and dV sums P^T dO, so the value row's total gradient is the sum of dO over the queries."""
+    rng = _rng(seed)
+    Q = rng.standard_normal((1, 1, N, D))
+    K = rng.standard_normal((1, 1, N, D))
+    V = np.tile(rng.standard_normal(D), (1, 1, N, 1))
+    W = rng.standard_normal((1, 1, N, D))
+    nb = N // block
+    idx = np.array([[[list(range(i + 1)) + [-1] * (nb - i - 1) for i in range(nb)]]], dtype=np.int32)
+    g = o.backward(Q, K, V, W, idx, block, True, 0.5)
+    assert np.abs(g["dQ"]).max() < 1e-12 and np.abs(g["dK"]).max() < 1e-12
+    assert np.allclose(g["dV"][0, 0].sum(axis=0), W[0, 0].sum(axis=0), atol=1e-10)
+
+
+def check_backward_gqa_sum(o, seed=28, N=64, block=16, D=8, topk=2):
+    """A KV head's dK and dV are the sums over its query heads of each head's own gradients."""
+    rng = _rng(seed)
+    Q = rng.standard_normal((1, 2, N, D))
+    K = rng.standard_normal((1, 1, N, D))
+    V = rng.standard_normal((1, 1, N, D))
+    W = rng.standard_normal((1, 2, N, D))
+    nb = N // block
+    idx = np.array([[[sorted(rng.choice(i + 1, size=min(topk, i + 1), replace=False).tolist())
+                      + [-1] * (topk - min(topk, i + 1)) for i in range(nb)]]], dtype=np.int32)
+    both = o.backward(Q, K, V, W, idx, block, True)
+    one = [o.backward(Q[:, h:h + 1], K, V, W[:, h:h + 1], idx, block, True) for h in range(2)]
+    assert np.allclose(both["dK"], one[0]["dK"] + one[1]["dK"], atol=1e-12)
+    assert np.allclose(both["dV"], one[0]["dV"] + one[1]["dV"], atol=1e-12)
+    assert np.allclose(both["dQ"][:, 1:], one[1]["dQ"], atol=1e-12)
+
+
 ALL_PINS = {
     "pyramid_means": check_pyramid_means,
     "query_summary": check_query_summary,
@@ -429,4 +511,9 @@ ALL_PINS = {
     "forced_budget_edges": check_forced_budget_edges,
     "capacity_pyramid_means": check_capacity_pyramid_means,
     "capacity_decode_equals_exact": check_capacity_decode_equals_exact,
+    "backward_finite_differences_causal": lambda o: check_backward_finite_differences(o, causal=True),
+    "backward_finite_differences_noncausal_gqa": lambda o: check_backward_finite_differences(
+        o, seed=29, causal=False, B=2, Hq=4, Hkv=2, nb=3, topk=2),
+    "backward_constant_values": check_backward_constant_values,
+    "backward_gqa_sum": check_backward_gqa_sum,
 }

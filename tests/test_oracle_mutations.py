@@ -22,6 +22,7 @@ _orig_node_value = po.node_value
 _orig_query_summary = po.query_summary
 _orig_merge = po.merge_partials
 _orig_level_sizes = po.level_sizes
+_orig_attend_backward = po.attend_backward
 
 
 def _drop_last_child(n_below, factor, c):
@@ -94,6 +95,33 @@ def _capacity_counts_spare_blocks(k_plane, block, factor, kv_len):
     return po.build_pyramid(k_plane, block, factor)
 
 
+def _backward_no_delta(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale, d_out):
+    # dS = P * dP (the row term rowsum(dO * O) dropped) is what dQ and dK then carry
+    dq, dk, dv = _orig_attend_backward(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale, d_out)
+    dq2, dk2, dv2 = _orig_attend_backward(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale,
+                                          np.zeros_like(d_out))
+    key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks]) if blocks else []
+    if len(key_pos) == 0:
+        return dq, dk, dv
+    q = q_rows.astype(np.float64)
+    kx = k_plane[key_pos].astype(np.float64)
+    vx = v_plane[key_pos].astype(np.float64)
+    s = scale * (q @ kx.T)
+    if causal:
+        s = np.where(np.asarray(key_pos)[None, :] > q_pos[:, None], -np.inf, s)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    ds = p * (d_out.astype(np.float64) @ vx.T)
+    dk_bad = np.zeros_like(dk)
+    np.add.at(dk_bad, key_pos, scale * (ds.T @ q))
+    return scale * (ds @ kx), dk_bad, dv
+
+
+def _backward_dk_unscaled(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale, d_out):
+    dq, dk, dv = _orig_attend_backward(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale, d_out)
+    return dq, dk / scale, dv
+
+
 def _one_level_too_many(n0, factor):
     sizes = [n0]
     while sizes[-1] >= factor:
@@ -118,6 +146,8 @@ MUTATIONS = {
     "sink repeated as the local block": ("forced_set", _forced_repeats_sink),
     "local block off by one": ("forced_set", _forced_local_is_previous_block),
     "capacity pyramid averages the spare rows": ("build_pyramid_capacity", _capacity_counts_spare_blocks),
+    "backward drops the row term of dS": ("attend_backward", _backward_no_delta),
+    "backward leaves the scale out of dK": ("attend_backward", _backward_dk_unscaled),
 }
 
 
