@@ -57,6 +57,9 @@ _sig = {
     "pisa_workspace_size": (ctypes.c_int, [_SP, _szp]),
     "pisa_build_pyramid": (ctypes.c_int, [_SP, _vp, _vp, _vp]),
     "pisa_append_pyramid": (ctypes.c_int, [_SP, _vp, _vp, ctypes.c_int32, _vp]),
+    "pisa_backward_workspace_size": (ctypes.c_int, [_SP, _szp]),
+    "pisa_sparse_attention_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                      ctypes.c_size_t, _vp]),
     "pisa_select_blocks": (ctypes.c_int, [_SP, _vp, _vp, _i32p, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "pisa_sparse_attention": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "pisa_forward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -271,6 +274,34 @@ def decode_attention_noalloc(shape: Shape, Q, K, V, idx, O=None, lse=True, strea
     _check(_lib.pisa_decode_attention_noalloc(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                               _ptr(O), _ptr(L), _stream(stream)), "pisa_decode_attention_noalloc")
     return O, L
+
+
+def backward_workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.pisa_backward_workspace_size(ctypes.byref(shape.c()), ctypes.byref(n)), "pisa_backward_workspace_size")
+    return n.value
+
+
+def sparse_attention_backward(shape: Shape, Q, K, V, O, lse, dO, idx, ws=None, dQ=None, dK=None, dV=None,
+                              stream=None):
+    """dQ, dK, dV of the sparse attention step for the selection `idx` (prefill)."""
+    torch = _torch()
+    B, Hq, N, D = shape.batch, shape.heads_q, shape.seq_q, shape.head_dim
+    for t, name in ((Q, "Q"), (O, "O"), (dO, "dO")):
+        _need(t, torch.bfloat16, (B, Hq, N, D), name)
+    for t, name in ((K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, (B, shape.heads_kv, shape.kv_rows, D), name)
+    _need(lse, torch.float32, (B, Hq, N), "lse")
+    _need(idx, torch.int32, (B, shape.hsel, shape.n_qblocks, shape.topk), "idx")
+    if ws is None:
+        ws = torch.zeros(backward_workspace_size(shape), dtype=torch.uint8, device=Q.device)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    _check(_lib.pisa_sparse_attention_backward(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                               _ptr(dO), _ptr(idx), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws), ws.numel(),
+                                               _stream(stream)), "pisa_sparse_attention_backward")
+    return dQ, dK, dV
 
 
 def check_status(ws, stream=None) -> tuple[int, int]:

@@ -342,6 +342,92 @@ pisa_status pisa_append_pyramid(const pisa_shape* shape, const void* K, float* p
     return pyramid_range(pl, K, pyramid, seq_kv_old / pl.blk, pl.n0, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Backward workspace: status word, Delta [B, Hq, N] fp32, list offsets [B, Hkv, n0 + 1] int32 and
+// list entries [B, Hkv, nqb * topk * g] int32.
+struct BwdLayout {
+    size_t delta, counts, entries, total;
+    int32_t max_entries;
+};
+
+static pisa_status bwd_layout(const Plan& pl, BwdLayout* w) {
+    if (pl.decode) return PISA_ERR_UNSUPPORTED;
+    if (pl.n0_cap != pl.n0) return PISA_ERR_INVALID_ARG;
+    if (pl.n0 + 1 > (227 * 1024) / 4) return PISA_ERR_UNSUPPORTED;  // list cursors of one plane in shared memory
+    const int64_t me = static_cast<int64_t>(pl.nqb) * pl.topk * pl.g;
+    if (me >= (int64_t(1) << 31)) return PISA_ERR_UNSUPPORTED;
+    w->max_entries = static_cast<int32_t>(me);
+    size_t o = kStatusBytes;
+    w->delta = o;
+    o = align256(o + static_cast<size_t>(pl.B) * pl.Hq * pl.N * sizeof(float));
+    w->counts = o;
+    o = align256(o + static_cast<size_t>(pl.B) * pl.Hkv * (pl.n0 + 1) * sizeof(int32_t));
+    w->entries = o;
+    o = align256(o + static_cast<size_t>(pl.B) * pl.Hkv * me * sizeof(int32_t));
+    w->total = o;
+    return PISA_OK;
+}
+
+pisa_status pisa_backward_workspace_size(const pisa_shape* shape, size_t* bytes) {
+    Plan pl;
+    pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    if (bytes == nullptr) return PISA_ERR_INVALID_ARG;
+    BwdLayout w;
+    if ((s = bwd_layout(pl, &w)) != PISA_OK) return s;
+    *bytes = w.total;
+    return PISA_OK;
+}
+
+pisa_status pisa_sparse_attention_backward(const pisa_shape* shape, const void* Q, const void* K, const void* V,
+                                           const void* O, const float* lse, const void* dO, const int32_t* idx,
+                                           void* dQ, void* dK, void* dV, void* ws, size_t ws_bytes,
+                                           pisa_stream_t stream) {
+    g_launches = 0;
+    Plan pl;
+    pisa_status s = make_plan(shape, &pl);
+    if (s != PISA_OK) return s;
+    BwdLayout w;
+    if ((s = bwd_layout(pl, &w)) != PISA_OK) return s;
+    const void* ptrs[] = {Q, K, V, O, lse, dO, idx, dQ, dK, dV};
+    for (const void* q : ptrs)
+        if (q == nullptr || !aligned16(q)) return PISA_ERR_INVALID_ARG;
+    if (ws == nullptr || !aligned16(ws)) return PISA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return PISA_ERR_WORKSPACE;
+    uint8_t* wb = static_cast<uint8_t*>(ws);
+    BwdParams p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q);
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.V = static_cast<const __nv_bfloat16*>(V);
+    p.O = static_cast<const __nv_bfloat16*>(O);
+    p.dO = static_cast<const __nv_bfloat16*>(dO);
+    p.lse = lse;
+    p.idx = idx;
+    p.dQ = static_cast<__nv_bfloat16*>(dQ);
+    p.dK = static_cast<__nv_bfloat16*>(dK);
+    p.dV = static_cast<__nv_bfloat16*>(dV);
+    p.delta = reinterpret_cast<float*>(wb + w.delta);
+    p.counts = reinterpret_cast<int32_t*>(wb + w.counts);
+    p.entries = reinterpret_cast<int32_t*>(wb + w.entries);
+    p.status = reinterpret_cast<uint32_t*>(wb);
+    p.Hq = pl.Hq;
+    p.Hkv = pl.Hkv;
+    p.g = pl.g;
+    p.N = pl.N;
+    p.n0 = pl.n0;
+    p.nqb = pl.nqb;
+    p.topk = pl.topk;
+    p.causal = pl.causal;
+    p.per_qhead = pl.per_qhead;
+    p.Hsel = pl.Hsel;
+    p.D = pl.D;
+    p.blk = pl.blk;
+    p.max_entries = w.max_entries;
+    p.scale = pl.scale;
+    p.scale_log2 = pl.scale * 1.4426950408889634f;
+    if (!launch_attn_backward(p, pl.B, reinterpret_cast<cudaStream_t>(stream), &g_launches)) return PISA_ERR_CUDA;
+    return PISA_OK;
+}
+
 static pisa_status check_budget(const Plan& pl, const int32_t* level_budget) {
     if (level_budget == nullptr) return PISA_OK;
     if (level_budget[0] != pl.topk) return PISA_ERR_INVALID_ARG;

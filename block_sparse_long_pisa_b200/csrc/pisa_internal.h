@@ -132,6 +132,26 @@ struct DecodeParams {
     float scale_log2;
 };
 
+struct BwdParams {
+    const __nv_bfloat16* Q;     // [B, Hq, N, D]
+    const __nv_bfloat16* K;     // [B, Hkv, N, D]
+    const __nv_bfloat16* V;
+    const __nv_bfloat16* O;     // forward output [B, Hq, N, D]
+    const __nv_bfloat16* dO;    // gradient of O
+    const float* lse;           // forward LSE [B, Hq, N] (natural log)
+    const int32_t* idx;         // [B, Hsel, nqb, topk]
+    __nv_bfloat16* dQ;          // [B, Hq, N, D]
+    __nv_bfloat16* dK;          // [B, Hkv, N, D]
+    __nv_bfloat16* dV;
+    float* delta;               // workspace [B, Hq, N]
+    int32_t* counts;            // workspace [B, Hkv, n0 + 1]: list offsets of every key block
+    int32_t* entries;           // workspace [B, Hkv, max_entries]: (query block * g + head in group)
+    uint32_t* status;
+    int32_t Hq, Hkv, g, N, n0, nqb, topk, causal, per_qhead, Hsel, D, blk;
+    int32_t max_entries;        // nqb * topk * g
+    float scale, scale_log2;
+};
+
 // ---------------------------------------------------------------- launchers (return false on launch error)
 
 bool launch_block_mean(const MeanParams& p, cudaStream_t st);
@@ -146,6 +166,7 @@ bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st
 pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
                                 cudaStream_t st, int32_t* launches);
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
+bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
 

@@ -197,6 +197,29 @@ PISA_API pisa_status pisa_sparse_attention(const pisa_shape *shape, const void *
                                   const void *V, const int32_t *idx, void *O, float *lse,
                                   void *ws, size_t ws_bytes, pisa_stream_t stream);
 
+/* Workspace bytes pisa_sparse_attention_backward needs for `shape` (prefill shapes only;
+ * PISA_ERR_UNSUPPORTED for decode). Host only. */
+PISA_API pisa_status pisa_backward_workspace_size(const pisa_shape *shape, size_t *bytes);
+
+/* Backward of step 3 through a fixed selection (PISA page, section "Ce que cela change pour
+ * vous": the sparse kernels also serve training; the block selection is a discrete choice and
+ * passes no gradient). With S = scale Q K^T over the selected keys, P = exp(S - LSE):
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),  dQ = scale dS K,  dK = scale dS^T Q,
+ * a KV head's dK and dV summing over all query rows (of all its query heads) that use each key.
+ *   Q, K, V, O : bf16 as in pisa_sparse_attention (O its output), device.
+ *   lse        : fp32 [batch, heads_q, seq_q], the forward's LSE, device.
+ *   dO         : bf16, same layout as O, device.
+ *   idx        : the selection the forward used (same rules on invalid entries).
+ *   dQ, dK, dV : bf16 outputs, the layouts of Q, K, V, device. Every element is written (keys
+ *                no query uses get 0).
+ *   ws         : >= pisa_backward_workspace_size bytes, 16-byte aligned, device.
+ * Prefill only (seq_q == seq_kv, no spare capacity); PISA_ERR_UNSUPPORTED otherwise.
+ * Deterministic: no atomics; every sum runs in a fixed order. Asynchronous on `stream`. */
+PISA_API pisa_status pisa_sparse_attention_backward(const pisa_shape *shape, const void *Q, const void *K,
+                                                    const void *V, const void *O, const float *lse,
+                                                    const void *dO, const int32_t *idx, void *dQ, void *dK,
+                                                    void *dV, void *ws, size_t ws_bytes, pisa_stream_t stream);
+
 /* Steps 1-3 in one call on one stream: pyramid and query summaries into the
  * workspace, selection, attention.
  *   idx_out : optional int32 [batch, Hsel, nQB, topk] copy of the selection
