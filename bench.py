@@ -461,6 +461,73 @@ def run_decode(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args, world, rank, local):
+    """Backward step of the sparse attention (dQ, dK, dV through the forward's selection).
+
+    Reported on its own line (not the forward's metric). Setup, outside the timed region: one
+    forward for O, LSE and the selection, and a seeded dO. Algorithmic work: 10 * D flops per
+    unmasked (query, key) pair (S, dP, dQ, dK and dV products once each; the kernels recompute
+    S and dP in both passes, 14 * D actual).
+    """
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = rank_workload(bench_workload(args), rank)
+    shape = pisa.Shape.of(w)
+    q, k, v = (workloads.device_tensor(w, t, dev) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, dev)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1000)
+    do = torch.randn(tuple(q.shape), generator=g).to(torch.bfloat16).to(dev)
+    bws = torch.zeros(pisa.backward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+    launches = [0]
+
+    def step():
+        pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx, ws=bws, dQ=dq, dK=dk, dV=dv)
+        launches[0] += pisa.last_launch_count()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches[0] = 0
+    clock = ClockSampler(local)
+    if rank == 0:
+        clock.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = clock.stop() if rank == 0 else None
+    pisa.raise_on_device_error(ws, "backward")
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+    pairs = pisa.attention_pairs(idx.cpu().numpy(), shape)
+    flops = 10.0 * w.head_dim * pairs
+    pk, how = peaks()
+    achieved = flops / (ms_step / 1e3) / 1e12
+    if rank != 0:
+        return
+    line = {
+        "metric": "sparse-attn backward tokens/s at N=128K (dQ, dK, dV through the forward's selection)",
+        "value": whole_job_tokens_per_s(w.batch * w.seq_q, world, ms_step),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy, bf16 RNE)", "config": config_dict(w, world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"], "flops_per_step": flops,
+                     "peak_source": f"{how} bf16 dense (burst)", "traffic": None},
+        "gpu_launches": launches[0], "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def scored_candidates(shape, sizes) -> int:
     """Candidates the descent scores for the whole problem (host count, no GPU data needed)."""
     f, K = shape.factor, shape.topk
@@ -487,6 +554,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS),
                     help="prefill workload to time (default: the N=128K GQA workload)")
     ap.add_argument("--seq", type=int, default=0, help="override the sequence length (smaller profiling cases)")
+    ap.add_argument("--backward", action="store_true", help="time the backward step instead of the forward")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.impl == "reference":
@@ -499,7 +567,9 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        if workloads.WORKLOADS[args.workload].decode:
+        if args.backward:
+            run_backward(args, world, rank, local)
+        elif workloads.WORKLOADS[args.workload].decode:
             run_decode(args, world, rank, local)
         else:
             run_gpu(args, world, rank, local)

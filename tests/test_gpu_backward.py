@@ -3,7 +3,7 @@
 The tolerance is relative to the largest gradient entry: the kernels round P and dS to bf16
 before the dV, dQ and dK products (relative error 2^-9 per term) and write bf16 outputs
 (another 2^-9), with fp32 accumulation; errors above 2 % of the largest entry, or a mean error
-above 0.3 % of it, mean a wrong term, not rounding.
+above 0.1 % of it, mean a wrong term, not rounding (measured on B200: at most 0.8 % and 0.02 %).
 """
 import numpy as np
 import pytest
@@ -21,7 +21,7 @@ CASES = {
     "mha-b128-causal": W("bwd-mha-b128", 1, 2, 2, 12 * 128, 12 * 128, 128, 128, 8, 4, 1, "clustered", 43),
     "mha-d64-b64-causal": W("bwd-mha-d64", 1, 3, 3, 17 * 64, 17 * 64, 64, 64, 4, 6, 1, "clustered", 44),
 }
-REL_MAX, REL_MEAN = 2e-2, 3e-3
+REL_MAX, REL_MEAN = 2e-2, 1e-3
 
 
 def _grads(w, cuda_device, per_qhead=False, forced=0):
