@@ -15,16 +15,19 @@
 //   bwd_dq_kernel      row-parallel: one CTA per (batch, query head, query
 //                      block), one warp per 16 rows; S and dP recomputed per
 //                      selected block with mma.sync (m16n8k16, bf16 in, fp32
-//                      accumulate), dQ kept in registers and written once.
+//                      accumulate), dQ kept in registers and written once. The
+//                      next block's K and V copy overlaps this block's MMAs.
 //   bwd_index_*        the inverse of the selection: for every (batch, KV head,
 //                      key block) the (query block, query head) pairs that
 //                      use it, in ascending order (count, scan, ordered fill),
 //                      so the column pass sums in a fixed order.
 //   bwd_dkdv_kernel    column-parallel: one CTA per (batch, KV head, key
 //                      block), one warp per 16 keys; S^T and dP^T recomputed
-//                      for every pair of the list, dK and dV kept in registers
-//                      and written once. No atomics anywhere: results are
-//                      deterministic.
+//                      for every pair of the list (the next pair's Q, dO copy
+//                      overlapping), dK and dV kept in registers and written
+//                      once. No atomics anywhere: results are deterministic.
+// This first version uses the warp-level mma.sync tensor path; on B200 it is
+// bound by that path's issue rate, not by memory.
 // Operand tiles sit in shared memory as [rows][D] bf16 with the 16-byte chunks
 // of a row XOR-swizzled by the row index, so ldmatrix reads are conflict-free.
 #include <cuda_bf16.h>
@@ -60,9 +63,9 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Byte offset of element (row, col) in a swizzled [rows][D] bf16 tile.
 template <int D>
@@ -142,8 +145,10 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(BLK * 2) bwd_dq_kernel(const BwdParams p) {
     constexpr int THREADS = BLK * 2;  // BLK / 16 warps
     extern __shared__ __align__(1024) uint8_t smem[];
-    const uint32_t sQ = smem_u32(smem), sO = sQ + BLK * D * 2, sK = sO + BLK * D * 2, sV = sK + BLK * D * 2;
-    int32_t* list = reinterpret_cast<int32_t*>(smem + 4 * BLK * D * 2);
+    constexpr uint32_t TILE = BLK * D * 2;
+    // Q, dO, then two stages of (K, V): the next selected block's copy overlaps this one's MMAs
+    const uint32_t sQ = smem_u32(smem), sO = sQ + TILE, sKV = sO + TILE;
+    int32_t* list = reinterpret_cast<int32_t*>(smem + 6 * TILE);
     __shared__ int s_n;
 
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -169,9 +174,16 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dq_kernel(const BwdParams p) {
     }
     load_tile<D, THREADS>(sQ, p.Q + qbase * D, BLK);
     load_tile<D, THREADS>(sO, p.dO + qbase * D, BLK);
-    cp_async_wait_all();
-    __syncthreads();
+    cp_async_commit();
+    __syncthreads();  // the block list is written
     const int nsel = s_n;
+    auto load_kv = [&](int u) {
+        const int64_t row = kbase + static_cast<int64_t>(list[u]) * BLK;
+        load_tile<D, THREADS>(sKV + (u & 1) * 2 * TILE, p.K + row * D, BLK);
+        load_tile<D, THREADS>(sKV + (u & 1) * 2 * TILE + TILE, p.V + row * D, BLK);
+        cp_async_commit();
+    };
+    if (nsel > 0) load_kv(0);
 
     const int r0 = warp * 16;
     const float c2 = p.scale_log2;
@@ -183,11 +195,14 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dq_kernel(const BwdParams p) {
 
     for (int u = 0; u < nsel; ++u) {
         const int j = list[u];
-        __syncthreads();  // the previous block's tiles are no longer read
-        load_tile<D, THREADS>(sK, p.K + (kbase + static_cast<int64_t>(j) * BLK) * D, BLK);
-        load_tile<D, THREADS>(sV, p.V + (kbase + static_cast<int64_t>(j) * BLK) * D, BLK);
-        cp_async_wait_all();
-        __syncthreads();
+        const uint32_t sK = sKV + (u & 1) * 2 * TILE, sV = sK + TILE;
+        if (u + 1 < nsel) {
+            load_kv(u + 1);  // its stage was last read in iteration u - 1, closed by the barrier below
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();  // this block's K, V (and, the first time, Q and dO) are in shared memory
         for (int kc = 0; kc < BLK; kc += kKC) {
             float s[kKC / 8][4], dp[kKC / 8][4];
 #pragma unroll
@@ -238,7 +253,9 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dq_kernel(const BwdParams p) {
                 }
             }
         }
+        __syncthreads();  // every warp is done with this stage before it is refilled
     }
+    cp_async_wait<0>();  // (no selected block: the Q and dO copies)
     // dQ = scale * (dS K), bf16
     const float sc = p.scale;
     __nv_bfloat16* dst = p.dQ + (qbase + r0) * D;
@@ -298,32 +315,45 @@ __global__ void __launch_bounds__(32) bwd_index_fill_kernel(const BwdParams p) {
     const int hper = p.per_qhead ? p.g : 1;                 // selection rows of this plane per query block
     const int mult = p.per_qhead ? 1 : p.g;                  // entries per selected block
     const int64_t n_cand = static_cast<int64_t>(p.nqb) * hper * p.topk;
-    for (int64_t c0 = 0; c0 < n_cand; c0 += 32) {
-        const int64_t c = c0 + lane;
-        int32_t j = -1;
-        int i = 0, hsub = 0;
-        if (c < n_cand) {
-            const int slot = static_cast<int>(c % p.topk);
-            hsub = static_cast<int>((c / p.topk) % hper);
-            i = static_cast<int>(c / (static_cast<int64_t>(p.topk) * hper));
-            const int hs = p.per_qhead ? kvh * p.g + hsub : kvh;
-            j = p.idx[((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i) * p.topk + slot];
-            if (!valid_block(p, j, i)) j = -1;
-        }
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, j);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        if (j >= 0) {
-            const int pos = cursor[j] + rank * mult;
-            if (p.per_qhead) {
-                out[pos] = i * p.g + hsub;
-            } else {
-                for (int e = 0; e < p.g; ++e) out[pos + e] = i * p.g + e;
+    constexpr int BATCH = 8;  // candidate loads in flight per lane
+    for (int64_t cb = 0; cb < n_cand; cb += 32 * BATCH) {
+        int32_t jb[BATCH];
+#pragma unroll
+        for (int q = 0; q < BATCH; ++q) {
+            const int64_t c = cb + q * 32 + lane;
+            jb[q] = -1;
+            if (c < n_cand) {
+                const int slot = static_cast<int>(c % p.topk);
+                const int hsub = static_cast<int>((c / p.topk) % hper);
+                const int i = static_cast<int>(c / (static_cast<int64_t>(p.topk) * hper));
+                const int hs = p.per_qhead ? kvh * p.g + hsub : kvh;
+                jb[q] = p.idx[((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i) * p.topk + slot];
             }
         }
-        __syncwarp();
-        // the highest-ranked lane of each key block moves its cursor past the chunk's entries
-        if (j >= 0 && (peers >> lane) == 1u) cursor[j] += (rank + 1) * mult;
-        __syncwarp();
+        for (int q = 0; q < BATCH; ++q) {
+            const int64_t c = cb + q * 32 + lane;
+            int32_t j = -1;
+            int i = 0, hsub = 0;
+            if (c < n_cand) {
+                hsub = static_cast<int>((c / p.topk) % hper);
+                i = static_cast<int>(c / (static_cast<int64_t>(p.topk) * hper));
+                j = valid_block(p, jb[q], i) ? jb[q] : -1;
+            }
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, j);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            if (j >= 0) {
+                const int pos = cursor[j] + rank * mult;
+                if (p.per_qhead) {
+                    out[pos] = i * p.g + hsub;
+                } else {
+                    for (int e = 0; e < p.g; ++e) out[pos + e] = i * p.g + e;
+                }
+            }
+            __syncwarp();
+            // the highest-ranked lane of each key block moves its cursor past the chunk's entries
+            if (j >= 0 && (peers >> lane) == 1u) cursor[j] += (rank + 1) * mult;
+            __syncwarp();
+        }
     }
 }
 
@@ -333,9 +363,10 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
     constexpr int THREADS = BLK * 2;
     extern __shared__ __align__(1024) uint8_t smem[];
-    const uint32_t sK = smem_u32(smem), sV = sK + BLK * D * 2, sQ = sV + BLK * D * 2, sO = sQ + BLK * D * 2;
-    float* s_lse = reinterpret_cast<float*>(smem + 4 * BLK * D * 2);
-    float* s_dlt = s_lse + BLK;
+    constexpr uint32_t TILE = BLK * D * 2;
+    // K, V, then two stages of (Q, dO, LSE, Delta): the next pair's copy overlaps this one's MMAs
+    constexpr uint32_t STAGE = 2 * TILE + 2 * BLK * 4;
+    const uint32_t sK = smem_u32(smem), sV = sK + TILE, sStage = sV + TILE;
 
     const int j = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -348,7 +379,21 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
 
     load_tile<D, THREADS>(sK, p.K + kbase * D, BLK);
     load_tile<D, THREADS>(sV, p.V + kbase * D, BLK);
-    cp_async_wait_all();
+    cp_async_commit();
+    auto load_pair = [&](int e) {
+        const int code = ent[e];
+        const int i = code / p.g, h = kvh * p.g + code % p.g;
+        const int64_t qbase = (static_cast<int64_t>(b) * p.Hq + h) * p.N + static_cast<int64_t>(i) * BLK;
+        const uint32_t st = sStage + ((e - e_lo) & 1) * STAGE;
+        load_tile<D, THREADS>(st, p.Q + qbase * D, BLK);
+        load_tile<D, THREADS>(st + TILE, p.dO + qbase * D, BLK);
+        for (int t = threadIdx.x; t < BLK / 4; t += THREADS) {  // 16-byte pieces of the row statistics
+            cp_async16(st + 2 * TILE + t * 16, p.lse + qbase + t * 4);
+            cp_async16(st + 2 * TILE + BLK * 4 + t * 16, p.delta + qbase + t * 4);
+        }
+        cp_async_commit();
+    };
+    if (e_hi > e_lo) load_pair(e_lo);
 
     const int r0 = warp * 16;  // this warp's keys in the block
     const float c2 = p.scale_log2;
@@ -359,18 +404,17 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
         for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
 
     for (int e = e_lo; e < e_hi; ++e) {
-        const int code = ent[e];
-        const int i = code / p.g, h = kvh * p.g + code % p.g;
-        const int64_t qbase = (static_cast<int64_t>(b) * p.Hq + h) * p.N + static_cast<int64_t>(i) * BLK;
-        __syncthreads();  // the previous pair's tiles are no longer read
-        load_tile<D, THREADS>(sQ, p.Q + qbase * D, BLK);
-        load_tile<D, THREADS>(sO, p.dO + qbase * D, BLK);
-        for (int t = threadIdx.x; t < BLK; t += THREADS) {
-            s_lse[t] = p.lse[qbase + t] * 1.4426950408889634f;
-            s_dlt[t] = p.delta[qbase + t];
+        const int i = ent[e] / p.g;
+        const uint32_t sQ = sStage + ((e - e_lo) & 1) * STAGE, sO = sQ + TILE;
+        const float* s_lse = reinterpret_cast<const float*>(smem + (sQ - sK) + 2 * TILE);
+        const float* s_dlt = s_lse + BLK;
+        if (e + 1 < e_hi) {
+            load_pair(e + 1);  // its stage was last read in iteration e - 1, closed by the barrier below
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        cp_async_wait_all();
-        __syncthreads();
+        __syncthreads();  // this pair's tiles (and, the first time, K and V) are in shared memory
         for (int qc = 0; qc < BLK; qc += kKC) {
             float s[kKC / 8][4], dp[kKC / 8][4];
 #pragma unroll
@@ -401,7 +445,7 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
                 for (int x = 0; x < 4; ++x) {
                     const int kr = r0 + g4 + (x >> 1) * 8;        // key in the block
                     const int qq = qc + n * 8 + 2 * t4 + (x & 1);  // query in its block
-                    float pv = fast_exp2(s[n][x] * c2 - s_lse[qq]);
+                    float pv = fast_exp2(s[n][x] * c2 - s_lse[qq] * 1.4426950408889634f);
                     if (p.causal && j == i && kr > qq) pv = 0.f;
                     s[n][x] = pv;
                     dp[n][x] = pv * (dp[n][x] - s_dlt[qq]);
@@ -430,7 +474,9 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
                 }
             }
         }
+        __syncthreads();  // every warp is done with this stage before it is refilled
     }
+    cp_async_wait<0>();  // (no pair: the K and V copies)
     const float sc = p.scale;
     __nv_bfloat16* dK = p.dK + (kbase + r0) * D;
     __nv_bfloat16* dV = p.dV + (kbase + r0) * D;
@@ -449,8 +495,8 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dkdv_kernel(const BwdParams p) {
 template <int D, int BLK>
 static bool launch_bwd_variant(const BwdParams& p, int32_t batch, cudaStream_t st) {
     const int threads = BLK * 2;
-    const size_t smem_dq = 4 * BLK * D * 2 + static_cast<size_t>(p.topk) * 4;
-    const size_t smem_kv = 4 * BLK * D * 2 + 2 * BLK * sizeof(float);
+    const size_t smem_dq = 6 * BLK * D * 2 + static_cast<size_t>(p.topk) * 4;
+    const size_t smem_kv = 6 * BLK * D * 2 + 4 * BLK * sizeof(float);
     if (cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_dq)) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
