@@ -27,11 +27,15 @@
 //
 // Per key group g and tile h:
 //   S[h] = Q_h K_g^T     tcgen05 (A = Q and B = K from shared memory), fp32 in TMEM
-//   softmax: P = exp2(S*c - m) against the running row max m, written as bf16
+//   softmax: P = exp2(S*c - m) against a reference row max m, written as bf16
 //            back into the TMEM columns of S already read (keys 0-63 into
-//            columns 0-31, keys 64-127 into columns 64-95). m moves only when a
-//            score exceeds it by more than 2^8; then that group is redone from
-//            the intact S with the new max and O and the row sums are rescaled
+//            columns 0-31, keys 64-127 into columns 64-95). m is the row max of
+//            the first group; it does not move, so the two warps of a row meet
+//            only in the first group and the epilogue. A row whose later
+//            scores exceed m by more than 2^16 marks the CTA, and the whole
+//            unit runs again in a second pass where m moves whenever a score
+//            exceeds it by more than 2^8 (that group is redone from the intact
+//            S with the new max, O and the row sums are rescaled)
 //   O[h] += P_h V_g      tcgen05 with A = P read from TMEM, B = V (MN-major)
 // Because P overwrites S, a tile's next Q.K^T waits for its P.V. With two
 // tiles the MMA lane issues Q.K^T(0, g), P.V(1, g-1), Q.K^T(1, g), P.V(0, g):
@@ -78,9 +82,18 @@ struct PrefillCfg {
     static_assert(SMEM < (1 << 18), "descriptor offsets assume shared addresses below 2^18");
 };
 
-// Lazy rescale threshold (log2 units): the running max is kept until a new
-// row max exceeds it by this much, so probabilities stay below 2^8.
+// First pass: every row keeps the maximum of its first key group as the
+// reference for all later groups, so the two warps of a row need not agree on
+// a new maximum per group. Probabilities then stay below 2^kFirstPassLimit;
+// a row whose scores exceed that (in log2 units) marks the CTA, which redoes
+// its unit in a second pass with the exact lazy rescale below.
+constexpr float kFirstPassLimit = 16.0f;
+// Second pass: the running max is kept until a new row max exceeds it by this
+// much (log2 units), so probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f;
+// Named barrier at which all roles learn whether a second pass runs (1..8
+// are the softmax warp pairs' barriers).
+constexpr uint32_t kPassBarrier = 15;
 
 template <int D, int BLK, int NM>
 __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
@@ -106,6 +119,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
     int32_t* s_nsel = reinterpret_cast<int32_t*>(tmem_slot + 1);
     int32_t* s_diag = s_nsel + 1;             // list position of the diagonal block i, -1 if absent
+    int32_t* s_retry = s_diag + 1;            // set when a row outgrew the first pass's reference
     int32_t* list = reinterpret_cast<int32_t*>(aux + 512);
 
     const int tid = threadIdx.x;
@@ -168,6 +182,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         if (lane == 0) {
             *s_nsel = cnt < C::MAX_LIST ? cnt : C::MAX_LIST;
             *s_diag = diag;
+            *s_retry = 0;
         }
     }
     tc_fence_before();
@@ -180,18 +195,28 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
 
     int issued_last = -1;  // producer lanes: last group whose copies they started
     bool issued_any_mma = false;
+    // Every role runs its loop over the key groups once, then all meet at kPassBarrier; if a
+    // softmax row marked the CTA, every role runs it once more (second pass, exact rescale).
+    // Ring slots and barrier phases follow the running group count gg = pass * ngroups + g.
+    auto second_pass = [&]() -> bool {
+        named_bar_sync(kPassBarrier, C::THREADS);
+        return *reinterpret_cast<volatile int32_t*>(s_retry) != 0;
+    };
 
     if (warp == C::PRODUCER_WARP) {
-        if (lane < 2 && ngroups > 0) {
-            const bool is_k = lane == 0;
-            const void* tmap = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
-            uint8_t* ring = is_k ? Ks : Vs;
-            uint64_t* full = is_k ? k_full : v_full;
-            uint64_t* empty = is_k ? k_empty : v_empty;
-            prefetch_tmap(tmap);
-            for (int g = 0; g < ngroups; ++g) {
-                const int st = g % C::NST, use = g / C::NST;
-                if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
+        const bool is_k = lane == 0;
+        const void* tmap = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+        uint8_t* ring = is_k ? Ks : Vs;
+        uint64_t* full = is_k ? k_full : v_full;
+        uint64_t* empty = is_k ? k_empty : v_empty;
+        bool ok = true;
+        if (lane < 2 && ngroups > 0) prefetch_tmap(tmap);
+        for (int pass = 0; pass < 2; ++pass) {
+            for (int g = 0; ok && lane < 2 && g < ngroups; ++g) {
+                const int gg = pass * ngroups + g;
+                const int st = gg % C::NST, use = gg / C::NST;
+                if (!(ok = mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))))
+                    break;
                 const int nb = min(C::GB, nsel - g * C::GB);
                 mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * BLK * D * 2));
                 for (int u = 0; u < nb; ++u) {
@@ -202,82 +227,92 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
                         tma_load_2d(ring + st * C::KG_BYTES + s * C::SUB + u * BLK * 128, tmap, s * 64, krow,
                                     full + st);
                 }
-                issued_last = g;
+                issued_last = gg;
             }
+            __syncwarp();
+            if (pass == 0 && !second_pass()) break;
         }
-        __syncwarp();
     } else if (warp == C::MMA_WARP) {
-        if (lane == 0 && ngroups > 0) {
-            // Operand descriptors are formed once; every tile the MMAs read lies at a fixed offset
-            // from these bases. The start-address field holds address / 16 in 14 bits, and shared
-            // memory ends below 2^18 bytes, so adding offset / 16 never carries out of the field.
-            const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
-            const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
-            const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), C::SUB, 1024);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
-            tc_fence_after();
-            // S[h] = Q_h K_g^T (after P.V of group g-1 on tile h has released the TMEM columns)
-            auto qk = [&](int g, int h) -> bool {
-                const int st = g % C::NST;
-                if (g > 0 && !mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x12u)) return false;
+        bool ok = true;
+        int g0 = 0;  // groups of earlier passes
+        for (int pass = 0; pass < 2; ++pass) {
+            g0 = pass * ngroups;
+            if (lane == 0 && ngroups > 0 && ok) {
+                // Operand descriptors are formed once; every tile the MMAs read lies at a fixed offset
+                // from these bases. The start-address field holds address / 16 in 14 bits, and shared
+                // memory ends below 2^18 bytes, so adding offset / 16 never carries out of the field.
+                const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
+                const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
+                const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), C::SUB, 1024);
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+                if (pass == 0) ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
                 tc_fence_after();
-                const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
-                const uint32_t idesc_qk = idesc_bf16_f32(128, ncols, 0, 0);
-                const uint32_t d_tmem = tm + C::S_COL + h * 128;
-                const uint64_t a0 = dq0 + static_cast<uint32_t>((h * C::DS * C::SUB) >> 4);
-                const uint64_t b0 = dk0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
+                // S[h] = Q_h K_g^T (after P.V of group g-1 on tile h has released the TMEM columns)
+                auto qk = [&](int g, int h) -> bool {
+                    const int gg = g0 + g;
+                    const int st = gg % C::NST;
+                    if (gg > 0 && !mbar_wait(pv_done + h, (gg - 1) & 1, p.status, detail_base | 0x12u)) return false;
+                    tc_fence_after();
+                    const int ncols = min(C::GB, nsel - g * C::GB) * BLK;
+                    const uint32_t idesc_qk = idesc_bf16_f32(128, ncols, 0, 0);
+                    const uint32_t d_tmem = tm + C::S_COL + h * 128;
+                    const uint64_t a0 = dq0 + static_cast<uint32_t>((h * C::DS * C::SUB) >> 4);
+                    const uint64_t b0 = dk0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = static_cast<uint32_t>(((ks / 4) * C::SUB + (ks % 4) * 32) >> 4);
-                    mma_bf16_ss(d_tmem, a0 + off, b0 + off, idesc_qk, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(s_full + h);
-                issued_any_mma = true;
-                return true;
-            };
-            // O[h] += P_h V_g (P in TMEM: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
-            auto pv = [&](int g, int h) -> bool {
-                const int st = g % C::NST;
-                if (!mbar_wait(p_full + h, g & 1, p.status, detail_base | 0x14u)) return false;
-                tc_fence_after();
-                const int nks = min(C::GB, nsel - g * C::GB) * BLK / 16;
-                const uint32_t d_tmem = tm + C::O_COL + h * D;
-                const uint32_t a_tmem = tm + C::S_COL + h * 128;
-                const uint64_t b0 = dv0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = static_cast<uint32_t>(((ks / 4) * C::SUB + (ks % 4) * 32) >> 4);
+                        mma_bf16_ss(d_tmem, a0 + off, b0 + off, idesc_qk, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full + h);
+                    issued_any_mma = true;
+                    return true;
+                };
+                // O[h] += P_h V_g (P in TMEM: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
+                auto pv = [&](int g, int h) -> bool {
+                    const int gg = g0 + g;
+                    const int st = gg % C::NST;
+                    if (!mbar_wait(p_full + h, gg & 1, p.status, detail_base | 0x14u)) return false;
+                    tc_fence_after();
+                    const int nks = min(C::GB, nsel - g * C::GB) * BLK / 16;
+                    const uint32_t d_tmem = tm + C::O_COL + h * D;
+                    const uint32_t a_tmem = tm + C::S_COL + h * 128;
+                    const uint64_t b0 = dv0 + static_cast<uint32_t>((st * C::KG_BYTES) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    if (ks < nks) {
-                        const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
-                        mma_bf16_ts(d_tmem, a_tmem + acol, b0 + static_cast<uint32_t>((ks * 16 * 128) >> 4), idesc_pv,
-                                    (g > 0 || ks > 0) ? 1u : 0u);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        if (ks < nks) {
+                            const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
+                            const uint32_t boff = static_cast<uint32_t>((ks * 16 * 128) >> 4);
+                            mma_bf16_ts(d_tmem, a_tmem + acol, b0 + boff, idesc_pv, (g > 0 || ks > 0) ? 1u : 0u);
+                        }
                     }
-                }
-                mma_commit(pv_done + h);
-                return true;
-            };
-            for (int g = 0; ok && g < ngroups; ++g) {
-                const int st = g % C::NST, ph = (g / C::NST) & 1;
-                if (!(ok = mbar_wait(k_full + st, ph, p.status, detail_base | 0x11u))) break;
-                if (!(ok = qk(g, 0))) break;
-                if (NM == 2) {
-                    if (g > 0) {
-                        // P.V(1, g-1) goes between the two Q.K^T of group g
-                        if (!(ok = pv(g - 1, 1))) break;
-                        mma_commit(v_empty + (g - 1) % C::NST);
+                    mma_commit(pv_done + h);
+                    return true;
+                };
+                for (int g = 0; ok && g < ngroups; ++g) {
+                    const int gg = g0 + g;
+                    const int st = gg % C::NST, ph = (gg / C::NST) & 1;
+                    if (!(ok = mbar_wait(k_full + st, ph, p.status, detail_base | 0x11u))) break;
+                    if (!(ok = qk(g, 0))) break;
+                    if (NM == 2) {
+                        if (g > 0) {
+                            // P.V(1, g-1) goes between the two Q.K^T of group g
+                            if (!(ok = pv(g - 1, 1))) break;
+                            mma_commit(v_empty + (gg - 1) % C::NST);
+                        }
+                        if (!(ok = qk(g, 1))) break;
                     }
-                    if (!(ok = qk(g, 1))) break;
+                    mma_commit(k_empty + st);
+                    if (!(ok = mbar_wait(v_full + st, ph, p.status, detail_base | 0x13u))) break;
+                    if (!(ok = pv(g, 0))) break;
+                    if (NM == 1) mma_commit(v_empty + st);
                 }
-                mma_commit(k_empty + st);
-                if (!(ok = mbar_wait(v_full + st, ph, p.status, detail_base | 0x13u))) break;
-                if (!(ok = pv(g, 0))) break;
-                if (NM == 1) mma_commit(v_empty + st);
+                if (ok && NM == 2) {
+                    if ((ok = pv(ngroups - 1, 1))) mma_commit(v_empty + (g0 + ngroups - 1) % C::NST);
+                }
             }
-            if (ok && NM == 2) {
-                if (pv(ngroups - 1, 1)) mma_commit(v_empty + (ngroups - 1) % C::NST);
-            }
+            __syncwarp();
+            if (pass == 0 && !second_pass()) break;
         }
-        __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax warps
         const int h = (warp / 4) % NM;
@@ -313,154 +348,173 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
         const uint64_t cs2 = f2_pack(cs, cs);
         float m_used = -INFINITY, l_part = 0.f;
         bool ok = true;
-        for (int g = 0; g < ngroups; ++g) {
-            const int nb = min(C::GB, nsel - g * C::GB);
-            const int ncols = nb * BLK;
-            const int mine = max(0, min(64, ncols - ch * 64));  // columns of this half that hold keys
-            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full + h, g & 1, p.status, detail_base | 0x20u));
-            tc_fence_after();
-            // first column of the diagonal block, 128 if this group does not hold it
-            const int diag_lo = (diag_pos >= 0 && diag_pos / C::GB == g) ? (diag_pos % C::GB) * BLK : 128;
-            const bool any_mask = ncols < 128 || diag_lo < 128;  // uniform across the CTA
-            uint32_t pk[32];                                     // this half's P, bf16 pairs
-            uint64_t sum2[2] = {0ull, 0ull};
-            float s_last = 0.f;  // raw score of this half's last column, whose TMEM cell the exchange reuses
-            // exp2 of one 32-column chunk against the reference max; returns the chunk's max x.
-            // TRACK, MASKED and PATCH are compile-time, so the unrolled pair loop has no branches
-            // and the compiler can interleave the sixteen independent pair chains. PATCH puts the
-            // saved last score back after an exchange has overwritten its cell.
-            auto chunk_exp = [&](int c, float m_ref, auto track_c, auto masked_c, auto patch_c) -> float {
-                constexpr bool TRACK = decltype(track_c)::value;
-                constexpr bool MASKED = decltype(masked_c)::value;
-                constexpr bool PATCH = decltype(patch_c)::value;
-                float sv[32];
-                tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                tmem_wait_ld();
-                if (c == 1) {
-                    if (PATCH)
-                        sv[31] = s_last;
-                    else
-                        s_last = sv[31];
-                }
-                if (MASKED) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = ch * 64 + c * 32 + k;
-                        if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
-                    }
-                }
-                const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
-                float xm = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int kk = c * 16 + k;
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
-                    if (TRACK) xm = fmax3(xm, x0, x1);
-                    const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
-                    sum2[k & 1] = f2_add(sum2[k & 1], e2);
-                    float e0, e1;
-                    f2_unpack(e2, e0, e1);
-                    pk[kk] = pack_bf16x2(e0, e1);
-                }
-                return xm;
-            };
-            // exponentials of this half against m_ref, after the exchange (saved last score restored)
-            auto exps_patched = [&](float m_ref) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    if (c * 32 < mine) {
-                        if (any_mask)
-                            chunk_exp(c, m_ref, std::false_type{}, std::true_type{}, std::true_type{});
+        int g_last = ngroups - 1;  // running index of the last group of the final pass
+        for (int pass = 0; pass < 2; ++pass) {
+            const bool exact = pass > 0;
+            const int g0 = pass * ngroups;
+            m_used = -INFINITY;
+            l_part = 0.f;
+            for (int g = 0; g < ngroups; ++g) {
+                const int gg = g0 + g;
+                const int nb = min(C::GB, nsel - g * C::GB);
+                const int ncols = nb * BLK;
+                const int mine = max(0, min(64, ncols - ch * 64));  // columns of this half that hold keys
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full + h, gg & 1, p.status, detail_base | 0x20u));
+                tc_fence_after();
+                // first column of the diagonal block, 128 if this group does not hold it
+                const int diag_lo = (diag_pos >= 0 && diag_pos / C::GB == g) ? (diag_pos % C::GB) * BLK : 128;
+                const bool any_mask = ncols < 128 || diag_lo < 128;  // uniform across the CTA
+                uint32_t pk[32];                                     // this half's P, bf16 pairs
+                uint64_t sum2[2] = {0ull, 0ull};
+                float s_last = 0.f;  // raw score of this half's last column, whose TMEM cell the exchange reuses
+                // exp2 of one 32-column chunk against the reference max; returns the chunk's max x.
+                // TRACK, MASKED and PATCH are compile-time, so the unrolled pair loop has no branches
+                // and the compiler can interleave the sixteen independent pair chains. PATCH puts the
+                // saved last score back after an exchange has overwritten its cell.
+                auto chunk_exp = [&](int c, float m_ref, auto track_c, auto masked_c, auto patch_c) -> float {
+                    constexpr bool TRACK = decltype(track_c)::value;
+                    constexpr bool MASKED = decltype(masked_c)::value;
+                    constexpr bool PATCH = decltype(patch_c)::value;
+                    float sv[32];
+                    tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                    tmem_wait_ld();
+                    if (c == 1) {
+                        if (PATCH)
+                            sv[31] = s_last;
                         else
-                            chunk_exp(c, m_ref, std::false_type{}, std::false_type{}, std::true_type{});
+                            s_last = sv[31];
                     }
-            };
-            float alpha = 1.0f, m_new = m_used;
-            if (g > 0) {
-                // fast path: probabilities against the running max m, kept while no score of the
-                // row (in either half) exceeds m by more than the rescale threshold
-                float xmax = -INFINITY;
+                    if (MASKED) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    if (c * 32 < mine)
-                        xmax = fmaxf(xmax, any_mask ? chunk_exp(c, m_used, std::true_type{}, std::true_type{},
-                                                                std::false_type{})
-                                                    : chunk_exp(c, m_used, std::true_type{}, std::false_type{},
-                                                                std::false_type{}));
-                const float xall = fmaxf(xmax, exchange(xmax));  // row max of s*c - m over both halves
-                if (__any_sync(0xFFFFFFFFu, xall > kRescaleThreshold)) {
-                    // the row max grew past the threshold: m moves up to it, O is rescaled, and the
-                    // exponentials are redone from S
-                    const bool resc = xall > kRescaleThreshold;
-                    m_new = resc ? m_used + xall : m_used;
-                    alpha = resc ? fast_exp2(-xall) : 1.0f;
-                    if (ok && __any_sync(0xFFFFFFFFu, resc)) {
-                        // O holds P.V of every earlier group (its completion preceded this S); this
-                        // warp rescales its half of the columns
-                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(pv_done + h, (g - 1) & 1, p.status, detail_base | 0x21u));
-                        if (ok) {
-                            tc_fence_after();
-#pragma unroll
-                            for (int c = 0; c < D / 32; ++c) {
-                                uint32_t o[16];
-                                const uint32_t addr = tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 16;
-                                tmem_ld16(addr, o);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                                tmem_st16(addr, o);
-                            }
+                        for (int k = 0; k < 32; ++k) {
+                            const int col = ch * 64 + c * 32 + k;
+                            if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
                         }
                     }
+                    const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+                    float xm = -INFINITY;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) sum2[k] = 0ull;
+                    for (int k = 0; k < 16; ++k) {
+                        const int kk = c * 16 + k;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(sv[2 * k], sv[2 * k + 1]), cs2, negm2), x0, x1);
+                        if (TRACK) xm = fmax3(xm, x0, x1);
+                        const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+                        sum2[k & 1] = f2_add(sum2[k & 1], e2);
+                        float e0, e1;
+                        f2_unpack(e2, e0, e1);
+                        pk[kk] = pack_bf16x2(e0, e1);
+                    }
+                    return xm;
+                };
+                // exponentials of this half against m_ref, after the exchange (saved last score restored)
+                auto exps_patched = [&](float m_ref) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        if (c * 32 < mine) {
+                            if (any_mask)
+                                chunk_exp(c, m_ref, std::false_type{}, std::true_type{}, std::true_type{});
+                            else
+                                chunk_exp(c, m_ref, std::false_type{}, std::false_type{}, std::true_type{});
+                        }
+                };
+                float alpha = 1.0f, m_new = m_used;
+                if (g > 0) {
+                    // fast path: probabilities against the running max m, kept while no score of the
+                    // row (in either half) exceeds m by more than the rescale threshold
+                    float xmax = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        if (c * 32 < mine)
+                            xmax = fmaxf(xmax, any_mask ? chunk_exp(c, m_used, std::true_type{}, std::true_type{},
+                                                                    std::false_type{})
+                                                        : chunk_exp(c, m_used, std::true_type{}, std::false_type{},
+                                                                    std::false_type{}));
+                    if (!exact) {
+                        // first pass: m stays the first group's row max; a row that outgrew it by more
+                        // than the limit sends the CTA to the second pass (this pass's P is discarded)
+                        if (valid && xmax > kFirstPassLimit) *reinterpret_cast<volatile int32_t*>(s_retry) = 1;
+                    } else {
+                        const float xall = fmaxf(xmax, exchange(xmax));  // row max of s*c - m over both halves
+                        if (__any_sync(0xFFFFFFFFu, xall > kRescaleThreshold)) {
+                            // the row max grew past the threshold: m moves up to it, O is rescaled, and the
+                            // exponentials are redone from S
+                            const bool resc = xall > kRescaleThreshold;
+                            m_new = resc ? m_used + xall : m_used;
+                            alpha = resc ? fast_exp2(-xall) : 1.0f;
+                            if (ok && __any_sync(0xFFFFFFFFu, resc)) {
+                                // O holds P.V of every earlier group (its completion preceded this S); this
+                                // warp rescales its half of the columns
+                                ok = __all_sync(0xFFFFFFFFu,
+                                                mbar_wait(pv_done + h, (gg - 1) & 1, p.status, detail_base | 0x21u));
+                                if (ok) {
+                                    tc_fence_after();
+#pragma unroll
+                                    for (int c = 0; c < D / 32; ++c) {
+                                        uint32_t o[16];
+                                        const uint32_t addr =
+                                            tm + lane_base + C::O_COL + h * D + ch * (D / 2) + c * 16;
+                                        tmem_ld16(addr, o);
+                                        tmem_wait_ld();
+#pragma unroll
+                                        for (int k = 0; k < 16; ++k)
+                                            o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                                        tmem_st16(addr, o);
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int k = 0; k < 2; ++k) sum2[k] = 0ull;
+                            exps_patched(m_new);
+                        }
+                    }
+                } else {
+                    // first group: the true row max, then the exponentials
+                    float mq[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) mq[q] = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        if (c * 32 < mine) {
+                            float sv[32];
+                            tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                            tmem_wait_ld();
+                            if (c == 1) s_last = sv[31];
+                            if (any_mask) {
+#pragma unroll
+                                for (int k = 0; k < 32; ++k) {
+                                    const int col = ch * 64 + c * 32 + k;
+                                    if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
+                                }
+                            }
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                mq[q] = fmax3(mq[q], sv[q], fmaxf(sv[8 + q], fmaxf(sv[16 + q], sv[24 + q])));
+                        }
+                    }
+                    const float mxs =
+                        fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7]))) * cs;
+                    m_new = fmaxf(mxs, exchange(mxs));
                     exps_patched(m_new);
                 }
-            } else {
-                // first group: the true row max, then the exponentials
-                float mq[8];
+                // P overwrites this half's S columns, already read: 64 scores -> 32 columns
 #pragma unroll
-                for (int q = 0; q < 8; ++q) mq[q] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    if (c * 32 < mine) {
-                        float sv[32];
-                        tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                        tmem_wait_ld();
-                        if (c == 1) s_last = sv[31];
-                        if (any_mask) {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                const int col = ch * 64 + c * 32 + k;
-                                if (col >= ncols || (col >= diag_lo && col - diag_lo > t)) sv[k] = -INFINITY;
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            mq[q] = fmax3(mq[q], sv[q], fmaxf(sv[8 + q], fmaxf(sv[16 + q], sv[24 + q])));
-                    }
-                }
-                const float mxs =
-                    fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], fmax3(mq[5], mq[6], mq[7]))) * cs;
-                m_new = fmaxf(mxs, exchange(mxs));
-                exps_patched(m_new);
+                for (int c = 0; c < 2; ++c)
+                    if (c * 32 < mine) tmem_st16(s_tmem + c * 16, *reinterpret_cast<uint32_t(*)[16]>(pk + c * 16));
+                float r0, r1;
+                f2_unpack(f2_add(sum2[0], sum2[1]), r0, r1);
+                l_part = l_part * alpha + (r0 + r1);
+                m_used = m_new;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(p_full + h);
             }
-            // P overwrites this half's S columns, already read: 64 scores -> 32 columns
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-                if (c * 32 < mine) tmem_st16(s_tmem + c * 16, *reinterpret_cast<uint32_t(*)[16]>(pk + c * 16));
-            float r0, r1;
-            f2_unpack(f2_add(sum2[0], sum2[1]), r0, r1);
-            l_part = l_part * alpha + (r0 + r1);
-            m_used = m_new;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full + h);
+            g_last = g0 + ngroups - 1;
+            if (pass == 0 && !second_pass()) break;
         }
         // ---------------------------------------------------------------- epilogue
         if (ok && ngroups > 0)
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(pv_done + h, (ngroups - 1) & 1, p.status, detail_base | 0x22u));
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(pv_done + h, g_last & 1, p.status, detail_base | 0x22u));
         const float l_sum = l_part + exchange(l_part);
         if (ok) {
             const int head = head0 + hh;
