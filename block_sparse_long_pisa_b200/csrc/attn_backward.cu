@@ -504,6 +504,7 @@ static bool launch_bwd_variant(const BwdParams& p, int32_t batch, cudaStream_t s
         return false;
     bwd_dq_kernel<D, BLK><<<dim3(p.nqb, p.Hq, batch), threads, smem_dq, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return false;
+    if (bwd_dkdv_tc_supported(p)) return launch_bwd_dkdv_tc(p, batch, st);
     bwd_dkdv_kernel<D, BLK><<<dim3(p.n0, p.Hkv, batch), threads, smem_kv, st>>>(p);
     return cudaGetLastError() == cudaSuccess;
 }

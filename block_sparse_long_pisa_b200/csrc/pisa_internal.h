@@ -34,6 +34,7 @@ enum : uint32_t {
     kKernAttnPrefill = 1,
     kKernAttnDecode = 2,
     kKernSelect = 3,
+    kKernAttnBackward = 4,
 };
 
 // Derived sizes of one problem (host side).
@@ -167,6 +168,10 @@ pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, co
                                 cudaStream_t st, int32_t* launches);
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
 bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
+// Backward column pass on the tensor cores (head dim 128, 64-key blocks); false when the shape is
+// another one or on a launch error.
+bool bwd_dkdv_tc_supported(const BwdParams& p);
+bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
 

@@ -20,6 +20,9 @@ CASES = {
     "gqa4-d64-noncausal": W("bwd-gqa4-d64", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 4, 0, "iid", 42),
     "mha-b128-causal": W("bwd-mha-b128", 1, 2, 2, 12 * 128, 12 * 128, 128, 128, 8, 4, 1, "clustered", 43),
     "mha-d64-b64-causal": W("bwd-mha-d64", 1, 3, 3, 17 * 64, 17 * 64, 64, 64, 4, 6, 1, "clustered", 44),
+    # head dim 128 with 64-key blocks: the column pass runs on the tensor-core (tcgen05) kernel
+    "gqa8-d128-noncausal": W("bwd-gqa8-d128", 2, 16, 2, 16 * 64, 16 * 64, 128, 64, 4, 6, 0, "clustered", 45),
+    "mha-d128-b64-causal": W("bwd-mha-d128", 1, 2, 2, 15 * 64, 15 * 64, 128, 64, 4, 4, 1, "iid", 46),
 }
 REL_MAX, REL_MEAN = 2e-2, 1e-3
 
@@ -68,10 +71,13 @@ def test_backward_per_qhead_and_forced(cuda_device):
     _close(dv, ref["dV"], "per-qhead dV")
 
 
-def test_backward_full_topk_is_dense_gradient(cuda_device):
-    """K = every block: the gradient of dense causal softmax attention."""
+@pytest.mark.parametrize("name", ["mha-d64-b64-causal", "mha-d128-b64-causal"])
+def test_backward_full_topk_is_dense_gradient(name, cuda_device):
+    """K = every block: the gradient of dense causal softmax attention (every key block's
+    inverse list then holds every later query block)."""
     import torch
-    w = CASES["mha-d64-b64-causal"].replace(topk=17)
+    w = CASES[name]
+    w = w.replace(topk=w.n_blocks)
     shape, (q, k, v, o, lse, do, idx), (dq, dk, dv) = _grads(w, cuda_device)
     nb = w.n_blocks
     full = np.full((w.batch, w.heads_kv, nb, nb), -1, dtype=np.int32)
