@@ -10,26 +10,30 @@
 // A KV head's dK and dV sum over all query rows (of all its query heads) whose
 // selection holds the key.
 //
-// Four launches:
+// Launches:
 //   bwd_delta_kernel   Delta per query row (fp32, workspace).
-//   bwd_dq_kernel      row-parallel: one CTA per (batch, query head, query
-//                      block), one warp per 16 rows; S and dP recomputed per
-//                      selected block with mma.sync (m16n8k16, bf16 in, fp32
-//                      accumulate), dQ kept in registers and written once. The
-//                      next block's K and V copy overlaps this block's MMAs.
 //   bwd_index_*        the inverse of the selection: for every (batch, KV head,
 //                      key block) the (query block, query head) pairs that
-//                      use it, in ascending order (count, scan, ordered fill),
+//                      use it, in ascending order (counts per range of query
+//                      blocks, scan, ordered fill of the ranges in parallel),
 //                      so the column pass sums in a fixed order.
+//   row pass (dQ) and column pass (dK, dV): for head dim 128 with 64-key
+//   blocks, the tcgen05/TMEM kernels of attn_backward_tc.cu; for the other
+//   shapes the two kernels below, on the warp-level mma.sync path:
+//   bwd_dq_kernel      row-parallel: one CTA per (batch, query head, query
+//                      block), one warp per 16 rows; S and dP recomputed per
+//                      selected block (m16n8k16, bf16 in, fp32 accumulate),
+//                      dQ kept in registers and written once. The next
+//                      block's K and V copy overlaps this block's MMAs.
 //   bwd_dkdv_kernel    column-parallel: one CTA per (batch, KV head, key
 //                      block), one warp per 16 keys; S^T and dP^T recomputed
 //                      for every pair of the list (the next pair's Q, dO copy
 //                      overlapping), dK and dV kept in registers and written
-//                      once. No atomics anywhere: results are deterministic.
-// This first version uses the warp-level mma.sync tensor path; on B200 it is
-// bound by that path's issue rate, not by memory.
-// Operand tiles sit in shared memory as [rows][D] bf16 with the 16-byte chunks
-// of a row XOR-swizzled by the row index, so ldmatrix reads are conflict-free.
+//                      once.
+// No atomics on any gradient: results are deterministic.
+// Operand tiles of the mma.sync kernels sit in shared memory as [rows][D]
+// bf16 with the 16-byte chunks of a row XOR-swizzled by the row index, so
+// ldmatrix reads are conflict-free.
 #include <cuda_bf16.h>
 
 #include "pisa_device.cuh"
@@ -273,56 +277,89 @@ __global__ void __launch_bounds__(BLK * 2) bwd_dq_kernel(const BwdParams p) {
 __global__ void __launch_bounds__(256) bwd_index_count_kernel(const BwdParams p, int64_t entries) {
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (t >= entries) return;
-    const int slot = static_cast<int>(t % p.topk);
     const int i = static_cast<int>((t / p.topk) % p.nqb);
     const int hs = static_cast<int>((t / (static_cast<int64_t>(p.topk) * p.nqb)) % p.Hsel);
     const int b = static_cast<int>(t / (static_cast<int64_t>(p.topk) * p.nqb * p.Hsel));
     const int32_t j = p.idx[t];
-    (void)slot;
     if (!valid_block(p, j, i)) return;
     const int kvh = p.per_qhead ? hs / p.g : hs;
-    atomicAdd(p.counts + (static_cast<int64_t>(b) * p.Hkv + kvh) * (p.n0 + 1) + j, p.per_qhead ? 1 : p.g);
+    const int64_t plane = static_cast<int64_t>(b) * p.Hkv + kvh;
+    atomicAdd(p.rcounts + (plane * p.nranges + i / p.rsize) * p.n0 + j, p.per_qhead ? 1 : p.g);
 }
 
-// One CTA (one warp) per (batch, KV head) plane: exclusive scan of the counts into list offsets,
-// then the entries in ascending (query block, query head) order. Equal key blocks within a chunk
-// of 32 candidates are ranked by lane (match.any), so the order is fixed.
-__global__ void __launch_bounds__(32) bwd_index_fill_kernel(const BwdParams p) {
-    extern __shared__ int32_t cursor[];  // [n0 + 1]
-    const int lane = threadIdx.x;
-    const int plane = blockIdx.x;  // b * Hkv + kvh
-    const int b = plane / p.Hkv, kvh = plane % p.Hkv;
+// One CTA per (batch, KV head) plane. Per key block j: the counts of the query-block ranges
+// become running sums (where each range's entries start inside j's list), the list lengths are
+// scanned into offsets (counts), and every range cursor is moved to its absolute position.
+__global__ void __launch_bounds__(256) bwd_index_scan_kernel(const BwdParams p) {
+    __shared__ int32_t part[256];
+    const int plane = blockIdx.x;
+    int32_t* rc = p.rcounts + static_cast<int64_t>(plane) * p.nranges * p.n0;
     int32_t* offs = p.counts + static_cast<int64_t>(plane) * (p.n0 + 1);
-    int32_t* out = p.entries + static_cast<int64_t>(plane) * p.max_entries;
-    // exclusive scan (counts -> offsets), chunk by chunk
-    int run = 0;
-    for (int c0 = 0; c0 <= p.n0; c0 += 32) {
-        const int c = c0 + lane;
-        const int v = c < p.n0 ? offs[c] : 0;
-        int x = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-            if (lane >= o) x += y;
+    const int n = p.n0 + 1;  // list lengths and the total
+    for (int j = threadIdx.x; j < p.n0; j += blockDim.x) {
+        int acc = 0;
+        for (int r = 0; r < p.nranges; ++r) {
+            const int c = rc[static_cast<int64_t>(r) * p.n0 + j];
+            rc[static_cast<int64_t>(r) * p.n0 + j] = acc;
+            acc += c;
         }
-        if (c <= p.n0) {
-            offs[c] = run + x - v;
-            cursor[c] = run + x - v;
-        }
-        run += __shfl_sync(0xFFFFFFFFu, x, 31);
+        offs[j] = acc;
     }
+    __syncthreads();
+    // exclusive scan of offs[0 .. n0] (offs[n0] taken as 0): each thread a contiguous segment
+    const int seg = (n + blockDim.x - 1) / blockDim.x;
+    const int lo = threadIdx.x * seg, hi = min(n, lo + seg);
+    int sum = 0;
+    for (int j = lo; j < hi; ++j) sum += j < p.n0 ? offs[j] : 0;
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int k = 0; k < static_cast<int>(blockDim.x); ++k) {
+            const int v = part[k];
+            part[k] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int run = part[threadIdx.x];
+    for (int j = lo; j < hi; ++j) {
+        const int v = j < p.n0 ? offs[j] : 0;
+        offs[j] = run;
+        run += v;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < p.n0; j += blockDim.x) {
+        const int off = offs[j];
+        for (int r = 0; r < p.nranges; ++r) rc[static_cast<int64_t>(r) * p.n0 + j] += off;
+    }
+}
+
+// One warp per (range of query blocks, plane): the range's entries in ascending (query block,
+// query head) order, starting at the cursors the scan left. Equal key blocks within a chunk of 32
+// candidates are ranked by lane (match.any), so the order is fixed.
+__global__ void __launch_bounds__(32) bwd_index_fill_kernel(const BwdParams p) {
+    extern __shared__ int32_t cursor[];  // [n0]
+    const int lane = threadIdx.x;
+    const int r = blockIdx.x, plane = blockIdx.y;  // plane = b * Hkv + kvh
+    const int b = plane / p.Hkv, kvh = plane % p.Hkv;
+    const int32_t* rc = p.rcounts + (static_cast<int64_t>(plane) * p.nranges + r) * p.n0;
+    int32_t* out = p.entries + static_cast<int64_t>(plane) * p.max_entries;
+    for (int j = lane; j < p.n0; j += 32) cursor[j] = rc[j];
     __syncwarp();
     const int hper = p.per_qhead ? p.g : 1;                 // selection rows of this plane per query block
     const int mult = p.per_qhead ? 1 : p.g;                  // entries per selected block
-    const int64_t n_cand = static_cast<int64_t>(p.nqb) * hper * p.topk;
+    const int i_lo = r * p.rsize, i_hi = min(p.nqb, i_lo + p.rsize);
+    const int64_t c_lo = static_cast<int64_t>(i_lo) * hper * p.topk;
+    const int64_t c_hi = static_cast<int64_t>(i_hi) * hper * p.topk;
     constexpr int BATCH = 8;  // candidate loads in flight per lane
-    for (int64_t cb = 0; cb < n_cand; cb += 32 * BATCH) {
+    for (int64_t cb = c_lo; cb < c_hi; cb += 32 * BATCH) {
         int32_t jb[BATCH];
 #pragma unroll
         for (int q = 0; q < BATCH; ++q) {
             const int64_t c = cb + q * 32 + lane;
             jb[q] = -1;
-            if (c < n_cand) {
+            if (c < c_hi) {
                 const int slot = static_cast<int>(c % p.topk);
                 const int hsub = static_cast<int>((c / p.topk) % hper);
                 const int i = static_cast<int>(c / (static_cast<int64_t>(p.topk) * hper));
@@ -334,7 +371,7 @@ __global__ void __launch_bounds__(32) bwd_index_fill_kernel(const BwdParams p) {
             const int64_t c = cb + q * 32 + lane;
             int32_t j = -1;
             int i = 0, hsub = 0;
-            if (c < n_cand) {
+            if (c < c_hi) {
                 hsub = static_cast<int>((c / p.topk) % hper);
                 i = static_cast<int>(c / (static_cast<int64_t>(p.topk) * hper));
                 j = valid_block(p, jb[q], i) ? jb[q] : -1;
@@ -502,8 +539,12 @@ static bool launch_bwd_variant(const BwdParams& p, int32_t batch, cudaStream_t s
         cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_kv)) != cudaSuccess)
         return false;
-    bwd_dq_kernel<D, BLK><<<dim3(p.nqb, p.Hq, batch), threads, smem_dq, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return false;
+    if (bwd_dq_tc_supported(p)) {
+        if (!launch_bwd_dq_tc(p, batch, st)) return false;
+    } else {
+        bwd_dq_kernel<D, BLK><<<dim3(p.nqb, p.Hq, batch), threads, smem_dq, st>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return false;
+    }
     if (bwd_dkdv_tc_supported(p)) return launch_bwd_dkdv_tc(p, batch, st);
     bwd_dkdv_kernel<D, BLK><<<dim3(p.n0, p.Hkv, batch), threads, smem_kv, st>>>(p);
     return cudaGetLastError() == cudaSuccess;
@@ -521,20 +562,23 @@ bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, in
             bwd_delta_kernel<128><<<grid, 256, 0, st>>>(p, rows);
         if (cudaGetLastError() != cudaSuccess) return false;
     }
-    // inverse of the selection
-    if (cudaMemsetAsync(p.counts, 0, static_cast<size_t>(batch) * p.Hkv * (p.n0 + 1) * sizeof(int32_t), st) !=
-        cudaSuccess)
+    // inverse of the selection: counts per (plane, query-block range, key block), scan, ordered fill
+    if (cudaMemsetAsync(p.rcounts, 0,
+                        static_cast<size_t>(batch) * p.Hkv * p.nranges * p.n0 * sizeof(int32_t), st) != cudaSuccess)
         return false;
     const int64_t cand = static_cast<int64_t>(batch) * p.Hsel * p.nqb * p.topk;
     bwd_index_count_kernel<<<static_cast<unsigned>((cand + 255) / 256), 256, 0, st>>>(p, cand);
     if (cudaGetLastError() != cudaSuccess) return false;
-    const size_t smem_fill = static_cast<size_t>(p.n0 + 1) * sizeof(int32_t);
+    bwd_index_scan_kernel<<<static_cast<unsigned>(batch * p.Hkv), 256, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return false;
+    const size_t smem_fill = static_cast<size_t>(p.n0) * sizeof(int32_t);
     if (cudaFuncSetAttribute(bwd_index_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_fill)) != cudaSuccess)
         return false;
-    bwd_index_fill_kernel<<<static_cast<unsigned>(batch * p.Hkv), 32, smem_fill, st>>>(p);
+    bwd_index_fill_kernel<<<dim3(static_cast<unsigned>(p.nranges), static_cast<unsigned>(batch * p.Hkv)), 32,
+                            smem_fill, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return false;
-    *launches += 3;
+    *launches += 4;
     bool ok;
     if (p.D == 128)
         ok = p.blk == 64 ? launch_bwd_variant<128, 64>(p, batch, st) : launch_bwd_variant<128, 128>(p, batch, st);

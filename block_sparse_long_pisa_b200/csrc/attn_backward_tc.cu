@@ -297,6 +297,363 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- row pass: dQ
+//
+// One CTA per (batch, selection row, query block, pair of query heads): 128 query rows (two
+// heads x 64 tokens; one head and 64 valid rows under per-query-head selection) that share the
+// block list. The selected blocks are taken in groups of 128 keys (two blocks), as in the
+// forward. Per group g:
+//   S = Q K_g^T, dP = dO V_g^T        tcgen05 SS, M = 128 rows, N = 128 keys, fp32 in TMEM
+//   dS = P (dP - Delta), P = exp(scale S - LSE)   (elementwise warps, written as bf16 over the
+//                                      S columns already read: keys 0-63 into columns 0-31,
+//                                      keys 64-127 into columns 64-95)
+//   dQ += dS K_g                       tcgen05 with A = dS from TMEM, B = K_g (MN-major)
+// dQ = scale dQ at the end. S is double-buffered in TMEM (S 2 x 128, dP 128, dQ 128 columns), so
+// group g+1's S and dP are formed while group g's dS is computed and used; the K ring has three
+// stages (K is read by S(g) and by dQ(g)), the V ring two.
+// Roles: warps 0-7 elementwise (two per row: keys 64 (w / 4) .. of each group; in the epilogue,
+// head-dim columns 64 (w / 4) ..), warp 8 producer (block list, Q and dO once, K lane 0, V
+// lane 1), warp 9 MMA issue and TMEM allocation.
+namespace {
+
+constexpr int kRD = 128;                       // head dim
+constexpr int kRB = 64;                        // block
+constexpr int kRDS = kRD / 64;
+constexpr uint32_t kRSub = 128 * 128;          // [128 rows x 128 B]
+constexpr uint32_t kRTile = kRDS * kRSub;      // Q, dO, or one 128-key K / V group: 32 KB
+constexpr int kRNstK = 3;
+constexpr int kRNstV = 2;
+constexpr uint32_t kROffQ = 0;
+constexpr uint32_t kROffO = kRTile;
+constexpr uint32_t kROffK = 2 * kRTile;
+constexpr uint32_t kROffV = kROffK + kRNstK * kRTile;
+constexpr uint32_t kROffAux = kROffV + kRNstV * kRTile;
+constexpr int kRMaxList = kMaxPrefillTopk;
+constexpr uint32_t kRAux = 256 + kRMaxList * 4;
+constexpr uint32_t kRSmem = 1024 + kROffAux + kRAux;
+constexpr uint32_t kRColS = 0;     // S / dS of buffer s at 128 s
+constexpr uint32_t kRColDP = 256;
+constexpr uint32_t kRColDQ = 384;
+constexpr int kREwThreads = 256;
+constexpr int kRProducerWarp = 8;
+constexpr int kRMmaWarp = 9;
+constexpr int kRThreads = 320;
+static_assert(kRSmem <= 232448, "shared memory budget");
+static_assert(kRSmem < (1 << 18), "descriptor start addresses below 2^18");
+
+}  // namespace
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const BwdParams p, const int gh, const int chunks) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* aux = base + kROffAux;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+    uint64_t* q_full = bars;                   // 1     Q and dO rows landed
+    uint64_t* k_full = q_full + 1;             // NstK
+    uint64_t* k_empty = k_full + kRNstK;       // NstK  S and dQ MMAs of the group done
+    uint64_t* v_full = k_empty + kRNstK;       // NstV
+    uint64_t* v_empty = v_full + kRNstV;       // NstV  dP MMAs of the group done
+    uint64_t* sdp_full = v_empty + kRNstV;     // 1     S and dP of the group in TMEM
+    uint64_t* dp_read = sdp_full + 1;          // 1     elementwise warps read S and dP (256 arrivals)
+    uint64_t* ds_ready = dp_read + 1;          // 2     dS of S buffer s in TMEM (256 arrivals)
+    uint64_t* dq_done = ds_ready + 2;          // 1     dQ MMAs of the group done
+    uint64_t* mma_final = dq_done + 1;         // 1     teardown: every MMA issued has completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
+    int32_t* s_nsel = reinterpret_cast<int32_t*>(tmem_slot + 1);
+    int32_t* s_diag = s_nsel + 1;
+    int32_t* list = reinterpret_cast<int32_t*>(aux + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = p.nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
+    const int hs = static_cast<int>(blockIdx.y) / chunks;
+    const int chunk = static_cast<int>(blockIdx.y) % chunks;
+    const int b = static_cast<int>(blockIdx.z);
+    const int kvh = p.per_qhead ? hs / p.g : hs;
+    const int head0 = p.per_qhead ? hs : kvh * p.g + chunk * gh;
+    const uint32_t detail_base = (kKernAttnBackward << 8) | 0x80u;
+
+    if (warp == kRProducerWarp && lane == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kRNstK; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < kRNstV; ++s) {
+            mbar_init(v_full + s, 1);
+            mbar_init(v_empty + s, 1);
+        }
+        mbar_init(sdp_full, 1);
+        mbar_init(dp_read, kREwThreads);
+        mbar_init(ds_ready, kREwThreads);
+        mbar_init(ds_ready + 1, kREwThreads);
+        mbar_init(dq_done, 1);
+        mbar_init(mma_final, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmdO);
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * gh * kRB * kRD * 2));
+        for (int hh = 0; hh < gh; ++hh) {
+            const int32_t qrow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
+                                                      static_cast<int64_t>(i) * kRB);
+#pragma unroll
+            for (int s = 0; s < kRDS; ++s) {
+                tma_load_2d(base + kROffQ + s * kRSub + hh * kRB * 128, &tmQ, s * 64, qrow, q_full);
+                tma_load_2d(base + kROffO + s * kRSub + hh * kRB * 128, &tmdO, s * 64, qrow, q_full);
+            }
+        }
+    }
+    if (warp == kRMmaWarp) tmem_alloc(tmem_slot, 512);
+    if (warp == kRProducerWarp) {
+        // compact the block row: eligible entries in order; the diagonal block's position
+        const int32_t* row = p.idx + ((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i) * p.topk;
+        int cnt = 0, diag = -1;
+        for (int t0 = 0; t0 < p.topk; t0 += 32) {
+            const int t = t0 + lane;
+            const int32_t jj = t < p.topk ? row[t] : -1;
+            const bool ok = jj >= 0 && jj < p.n0 && (!p.causal || jj <= i);
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
+            const int pos = cnt + __popc(m & ((1u << lane) - 1u));
+            if (ok && pos < kRMaxList) list[pos] = jj;
+            const uint32_t md = __ballot_sync(0xFFFFFFFFu, p.causal && ok && jj == i && pos < kRMaxList);
+            if (diag < 0 && md != 0u) diag = __shfl_sync(0xFFFFFFFFu, pos, __ffs(md) - 1);
+            cnt += __popc(m);
+        }
+        if (lane == 0) {
+            *s_nsel = cnt < kRMaxList ? cnt : kRMaxList;
+            *s_diag = diag;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const int nsel = *s_nsel;
+    const int ngroups = (nsel + 1) / 2;
+    const int diag_pos = *s_diag;
+
+    int issued_last = -1;
+    if (warp == kRProducerWarp) {
+        if (lane < 2 && ngroups > 0) {
+            const bool is_k = lane == 0;
+            const void* tmap = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+            uint8_t* ring = base + (is_k ? kROffK : kROffV);
+            uint64_t* full = is_k ? k_full : v_full;
+            uint64_t* empty = is_k ? k_empty : v_empty;
+            const int nst = is_k ? kRNstK : kRNstV;
+            prefetch_tmap(tmap);
+            for (int g = 0; g < ngroups; ++g) {
+                const int st = g % nst, use = g / nst;
+                if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
+                const int nb = min(2, nsel - 2 * g);
+                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * kRB * kRD * 2));
+                for (int u = 0; u < nb; ++u) {
+                    const int32_t krow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N +
+                                                              static_cast<int64_t>(list[2 * g + u]) * kRB);
+#pragma unroll
+                    for (int s = 0; s < kRDS; ++s)
+                        tma_load_2d(ring + st * kRTile + s * kRSub + u * kRB * 128, tmap, s * 64, krow, full + st);
+                }
+                issued_last = g;
+            }
+        }
+        __syncwarp();
+    } else if (warp == kRMmaWarp) {
+        if (lane == 0 && ngroups > 0) {
+            const uint32_t sQ = smem_u32(base + kROffQ), sO = smem_u32(base + kROffO);
+            const uint32_t sK = smem_u32(base + kROffK), sV = smem_u32(base + kROffV);
+            constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kRD, 0, 1);
+            bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
+            auto ncols_of = [&](int g) { return min(2, nsel - 2 * g) * kRB; };
+            // dP(g) = dO V_g^T into the dP columns (after the elementwise warps read dP(g-1))
+            auto issue_dp = [&](int g) -> bool {
+                const int st = g % kRNstV;
+                if (!mbar_wait(v_full + st, (g / kRNstV) & 1, p.status, detail_base | 0x11u)) return false;
+                if (g > 0 && !mbar_wait(dp_read, (g - 1) & 1, p.status, detail_base | 0x12u)) return false;
+                tc_fence_after();
+                const uint32_t id = idesc_bf16_f32(128, ncols_of(g), 0, 0);
+#pragma unroll
+                for (int ks = 0; ks < kRD / 16; ++ks) {
+                    const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
+                    mma_bf16_ss(tm + kRColDP, smem_desc_sw128(sO + off, 16, 1024),
+                                smem_desc_sw128(sV + st * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(v_empty + st);
+                return true;
+            };
+            // S(g) = Q K_g^T into S buffer g % 2 (after dQ(g-2) read the dS it held)
+            auto issue_s = [&](int g) -> bool {
+                const int st = g % kRNstK;
+                if (!mbar_wait(k_full + st, (g / kRNstK) & 1, p.status, detail_base | 0x13u)) return false;
+                if (g > 1 && !mbar_wait(dq_done, (g - 2) & 1, p.status, detail_base | 0x14u)) return false;
+                tc_fence_after();
+                const uint32_t id = idesc_bf16_f32(128, ncols_of(g), 0, 0);
+#pragma unroll
+                for (int ks = 0; ks < kRD / 16; ++ks) {
+                    const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
+                    mma_bf16_ss(tm + kRColS + 128 * (g % 2), smem_desc_sw128(sQ + off, 16, 1024),
+                                smem_desc_sw128(sK + st * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(sdp_full);
+                return true;
+            };
+            // dQ += dS(g) K_g (dS in TMEM: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
+            auto issue_dq = [&](int g) -> bool {
+                const int st = g % kRNstK;
+                if (!mbar_wait(ds_ready + g % 2, (g / 2) & 1, p.status, detail_base | 0x15u)) return false;
+                tc_fence_after();
+                const int nks = ncols_of(g) / 16;
+                const uint32_t a_tmem = tm + kRColS + 128 * (g % 2);
+                const uint64_t b0 = smem_desc_sw128(sK + st * kRTile, kRSub, 1024);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    if (ks < nks) {
+                        const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
+                        const uint32_t boff = static_cast<uint32_t>((ks * 16 * 128) >> 4);
+                        mma_bf16_ts(tm + kRColDQ, a_tmem + acol, b0 + boff, idesc_dq, (g > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit(dq_done);
+                mma_commit(k_empty + st);
+                return true;
+            };
+            // dP(g+1) and S(g+1) go ahead of dQ(g), so the tensor pipe forms the next group's
+            // scores while the elementwise warps work on this one
+            if (ok) ok = issue_dp(0) && issue_s(0);
+            for (int g = 0; ok && g < ngroups; ++g) {
+                if (g + 1 < ngroups && !(ok = issue_dp(g + 1) && issue_s(g + 1))) break;
+                ok = issue_dq(g);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- elementwise warps
+        const int q = warp % 4, ch = warp / 4;  // TMEM lane quadrant; keys 64 ch .. of each group
+        const int r = q * 32 + lane;            // row of the tile
+        const bool valid = r < gh * kRB;
+        const int hh = valid ? r / kRB : 0, t = r % kRB;
+        const int64_t grow = (static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N + static_cast<int64_t>(i) * kRB + t;
+        const float lse2 = p.lse[grow] * 1.4426950408889634f;
+        const float dlt = p.delta[grow];
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const float c2 = p.scale_log2;
+        bool ok = true;
+        for (int g = 0; g < ngroups; ++g) {
+            const int ncols = min(2, nsel - 2 * g) * kRB;
+            const bool mine = ch * 64 < ncols;  // this half of the group holds keys
+            // first column of the diagonal block in this group (128: not here)
+            const int diag_lo = (diag_pos >= 0 && diag_pos / 2 == g) ? (diag_pos % 2) * kRB : 128;
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sdp_full, g & 1, p.status, detail_base | 0x20u));
+            tc_fence_after();
+            const uint32_t s_col = tm + lane_base + kRColS + 128 * (g % 2) + 64 * ch;
+            uint32_t pk[32];
+            if (mine) {
+                uint32_t sv[64], dv[64];
+                tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                tmem_ld32(tm + lane_base + kRColDP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(dv));
+                tmem_ld32(tm + lane_base + kRColDP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(dp_read);  // the dP columns may be overwritten
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int c0 = ch * 64 + 2 * k;  // key column in the group
+                    const bool m0 = !valid || (c0 >= diag_lo && c0 - diag_lo > t);
+                    const bool m1 = !valid || (c0 + 1 >= diag_lo && c0 + 1 - diag_lo > t);
+                    const float p0 = fast_exp2(__uint_as_float(sv[2 * k]) * c2 - lse2);
+                    const float p1 = fast_exp2(__uint_as_float(sv[2 * k + 1]) * c2 - lse2);
+                    const float d0 = m0 ? 0.f : p0 * (__uint_as_float(dv[2 * k]) - dlt);
+                    const float d1 = m1 ? 0.f : p1 * (__uint_as_float(dv[2 * k + 1]) - dlt);
+                    pk[k] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(s_col, *reinterpret_cast<uint32_t(*)[16]>(pk));
+                tmem_st16(s_col + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+                tmem_wait_st();
+            } else {
+                mbar_arrive(dp_read);
+            }
+            tc_fence_before();
+            mbar_arrive(ds_ready + g % 2);
+        }
+        // ---------------------------------------------------------------- epilogue
+        // dQ(ngroups - 1) done; phase by phase, since dq_done may still be one group behind
+        for (int g = max(0, ngroups - 2); ok && g < ngroups; ++g)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(dq_done, g & 1, p.status, detail_base | 0x22u));
+        tc_fence_after();
+        if (ok && valid) {
+            const float sc = p.scale;
+            uint4* dst = reinterpret_cast<uint4*>(p.dQ + grow * kRD + ch * 64);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o[32];
+                if (ngroups > 0) {
+                    tmem_ld32(tm + lane_base + kRColDQ + ch * 64 + c * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) o[x] = 0u;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint32_t v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        v[e] = pack_bf16x2(__uint_as_float(o[8 * k + 2 * e]) * sc,
+                                           __uint_as_float(o[8 * k + 2 * e + 1]) * sc);
+                    dst[c * 4 + k] = make_uint4(v[0], v[1], v[2], v[3]);
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncthreads();
+    if (warp == kRProducerWarp && lane < 2) {
+        uint64_t* full = lane == 0 ? k_full : v_full;
+        const int nst = lane == 0 ? kRNstK : kRNstV;
+        for (int g = max(0, issued_last - nst + 1); g <= issued_last; ++g)
+            mbar_wait(full + g % nst, (g / nst) & 1, p.status, detail_base | 0x30u);
+        if (lane == 0) mbar_wait(q_full, 0, p.status, detail_base | 0x31u);
+    }
+    if (warp == kRMmaWarp && lane == 0 && ngroups > 0) {
+        // every MMA issued (all of them, or what an error left) completes before TMEM is freed
+        mma_commit(mma_final);
+        mbar_wait(mma_final, 0, p.status, detail_base | 0x32u);
+    }
+    __syncthreads();
+    if (warp == kRMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+bool bwd_dq_tc_supported(const BwdParams& p) { return p.D == kRD && p.blk == kRB && p.topk <= kRMaxList; }
+
+bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
+    if (!bwd_dq_tc_supported(p)) return false;
+    CUtensorMap tq, tdo, tk, tv;
+    const int64_t qrows = static_cast<int64_t>(batch) * p.Hq * p.N;
+    const int64_t krows = static_cast<int64_t>(batch) * p.Hkv * p.N;
+    if (!make_tmap_2d(&tq, p.Q, qrows, kRD, kRB) || !make_tmap_2d(&tdo, p.dO, qrows, kRD, kRB) ||
+        !make_tmap_2d(&tk, p.K, krows, kRD, kRB) || !make_tmap_2d(&tv, p.V, krows, kRD, kRB))
+        return false;
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kRSmem)) != cudaSuccess)
+            return false;
+        configured = true;
+    }
+    const int gsel = p.per_qhead ? 1 : p.g;
+    const int gh = gsel % 2 == 0 ? 2 : 1;  // two heads fill the 128 rows; else one head (64 rows)
+    const int chunks = gsel / gh;
+    bwd_dq_tc_kernel<<<dim3(p.nqb, p.Hsel * chunks, batch), kRThreads, kRSmem, st>>>(tq, tdo, tk, tv, p, gh, chunks);
+    return cudaGetLastError() == cudaSuccess;
+}
+
 bool bwd_dkdv_tc_supported(const BwdParams& p) { return p.D == kTD && p.blk == kTB; }
 
 bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {

@@ -342,11 +342,13 @@ pisa_status pisa_append_pyramid(const pisa_shape* shape, const void* K, float* p
     return pyramid_range(pl, K, pyramid, seq_kv_old / pl.blk, pl.n0, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Backward workspace: status word, Delta [B, Hq, N] fp32, list offsets [B, Hkv, n0 + 1] int32 and
-// list entries [B, Hkv, nqb * topk * g] int32.
+// Backward workspace: status word, Delta [B, Hq, N] fp32, list offsets [B, Hkv, n0 + 1] int32,
+// list entries [B, Hkv, nqb * topk * g] int32 and per-range counts / cursors [B, Hkv, R, n0] int32
+// (the inverse lists are filled by R ranges of query blocks in parallel).
+constexpr int32_t kFillRanges = 32;
 struct BwdLayout {
-    size_t delta, counts, entries, total;
-    int32_t max_entries;
+    size_t delta, counts, entries, rcounts, total;
+    int32_t max_entries, nranges, rsize;
 };
 
 static pisa_status bwd_layout(const Plan& pl, BwdLayout* w) {
@@ -363,6 +365,10 @@ static pisa_status bwd_layout(const Plan& pl, BwdLayout* w) {
     o = align256(o + static_cast<size_t>(pl.B) * pl.Hkv * (pl.n0 + 1) * sizeof(int32_t));
     w->entries = o;
     o = align256(o + static_cast<size_t>(pl.B) * pl.Hkv * me * sizeof(int32_t));
+    w->rsize = (pl.nqb + kFillRanges - 1) / kFillRanges;
+    w->nranges = (pl.nqb + w->rsize - 1) / w->rsize;
+    w->rcounts = o;
+    o = align256(o + static_cast<size_t>(pl.B) * pl.Hkv * w->nranges * pl.n0 * sizeof(int32_t));
     w->total = o;
     return PISA_OK;
 }
@@ -408,6 +414,9 @@ pisa_status pisa_sparse_attention_backward(const pisa_shape* shape, const void* 
     p.delta = reinterpret_cast<float*>(wb + w.delta);
     p.counts = reinterpret_cast<int32_t*>(wb + w.counts);
     p.entries = reinterpret_cast<int32_t*>(wb + w.entries);
+    p.rcounts = reinterpret_cast<int32_t*>(wb + w.rcounts);
+    p.nranges = w.nranges;
+    p.rsize = w.rsize;
     p.status = reinterpret_cast<uint32_t*>(wb);
     p.Hq = pl.Hq;
     p.Hkv = pl.Hkv;

@@ -147,9 +147,11 @@ struct BwdParams {
     float* delta;               // workspace [B, Hq, N]
     int32_t* counts;            // workspace [B, Hkv, n0 + 1]: list offsets of every key block
     int32_t* entries;           // workspace [B, Hkv, max_entries]: (query block * g + head in group)
+    int32_t* rcounts;           // workspace [B, Hkv, nranges, n0]: per query-block range, then its list cursors
     uint32_t* status;
     int32_t Hq, Hkv, g, N, n0, nqb, topk, causal, per_qhead, Hsel, D, blk;
     int32_t max_entries;        // nqb * topk * g
+    int32_t nranges, rsize;     // the inverse lists are filled by ranges of rsize query blocks
     float scale, scale_log2;
 };
 
@@ -172,6 +174,9 @@ bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, in
 // another one or on a launch error.
 bool bwd_dkdv_tc_supported(const BwdParams& p);
 bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
+// Backward row pass (dQ) on the tensor cores, same shapes.
+bool bwd_dq_tc_supported(const BwdParams& p);
+bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
 
