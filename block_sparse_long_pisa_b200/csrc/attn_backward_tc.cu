@@ -7,6 +7,7 @@
 // time: a tile of 128 query rows. Per tile, with the forward's LSE and
 // Delta = rowsum(dO * O):
 //   S  = Q K_j^T,  dP = dO V_j^T            tcgen05, M = 128 rows, N = 64 keys, fp32 in TMEM
+//                                           (separate barriers: P is computed while dP forms)
 //   P  = exp(scale S - LSE),  dS = P (dP - Delta)   (elementwise warps, bf16 into shared memory)
 //   dV_j^T += dO^T P,  dK_j^T += Q^T dS     tcgen05, M = 128 (head dim), N = 64 keys, K = 128 rows
 // dK = scale dK_j. The two accumulators stay in TMEM for the whole list and are written once, so
@@ -14,7 +15,9 @@
 //
 // A 64-wide operand costs a tcgen05 MMA as much as a 128-wide one on this part (measured: M128
 // N64 and M64 N128 both take the cycles of M128 N128), so these MMAs run at half the peak rate;
-// a 64-key block leaves no 128-wide dimension here except the rows and the head dim.
+// a 64-key block leaves no 128-wide dimension here except the rows and the head dim. Per tile
+// the MMAs read 192 KB of shared memory (6 KB each), the copies write 64 KB and P, dS 32 KB:
+// shared-memory bandwidth (128 B per clock) bounds the pass near 2,250 cycles per tile.
 //
 // Roles: warps 0-7 elementwise (thread = query row = TMEM lane of quadrant w % 4, keys 32 (w / 4)
 // onwards; in the epilogue, head-dim lane), warp 8 TMA producer (K_j and V_j once, then Q and dO
@@ -69,8 +72,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* kv_full = bars;                 // 1    K_j and V_j landed
     uint64_t* qo_full = kv_full + 1;          // kNst Q and dO rows of the tile landed
     uint64_t* qo_empty = qo_full + kNst;      // kNst dV, dK MMAs of the tile done: Q/dO stage and P/dS free
-    uint64_t* sdp_full = qo_empty + kNst;     // kNst S and dP of the tile in TMEM
-    uint64_t* sdp_read = sdp_full + kNst;     // kNst the elementwise warps read S and dP (256 arrivals)
+    uint64_t* s_full = qo_empty + kNst;       // kNst S of the tile in TMEM
+    uint64_t* dp_full = s_full + kNst;        // kNst dP of the tile in TMEM
+    uint64_t* sdp_read = dp_full + kNst;      // kNst the elementwise warps read S and dP (256 arrivals)
     uint64_t* p_ready = sdp_read + kNst;      // kNst P and dS in shared memory (256 arrivals)
     uint64_t* mma_final = p_ready + kNst;     // 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
@@ -96,7 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kNst; ++s) {
             mbar_init(qo_full + s, 1);
             mbar_init(qo_empty + s, 1);
-            mbar_init(sdp_full + s, 1);
+            mbar_init(s_full + s, 1);
+            mbar_init(dp_full + s, 1);
             mbar_init(sdp_read + s, kEwThreads);
             mbar_init(p_ready + s, kEwThreads);
         }
@@ -161,13 +166,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ss(tm + kColS + 64 * st, smem_desc_sw128(sQ + oa, 16, 1024),
                                     smem_desc_sw128(sK + ob, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                     }
+                    mma_commit(s_full + st);  // the exponentials start while dP is formed
 #pragma unroll
                     for (int ks = 0; ks < kTD / 16; ++ks) {
                         const uint32_t oa = (ks / 4) * kSub + (ks % 4) * 32, ob = (ks / 4) * kKSub + (ks % 4) * 32;
                         mma_bf16_ss(tm + kColDP + 64 * st, smem_desc_sw128(sO + oa, 16, 1024),
                                     smem_desc_sw128(sV + ob, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                     }
-                    mma_commit(sdp_full + st);
+                    mma_commit(dp_full + st);
                 }
                 // dV^T += dO^T P and dK^T += Q^T dS: the head dim is M (two 64-column tiles LBO
                 // apart), the 128 rows are K (16 per MMA), the keys N
@@ -216,26 +222,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float dlt = p.delta[row];
             // keys from mask_from on are masked (causal diagonal block), all of them for a padding row
             const int mask_from = !valid ? 0 : ((p.causal && i == j) ? tr + 1 : kTB);
-            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sdp_full + st, ph, p.status, detail_base | 0x20u));
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full + st, ph, p.status, detail_base | 0x20u));
             tc_fence_after();
             uint32_t pk[16], dk[16];  // P and dS of this thread's 32 keys, bf16 pairs
             {
-                uint32_t sv[32], dv[32];
+                float pv[32];
+                uint32_t sv[32];
                 tmem_ld32(tm + lane_base + kColS + 64 * st + 32 * ch, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const float e = fast_exp2(__uint_as_float(sv[k]) * c2 - lse2);
+                    pv[k] = 32 * ch + k >= mask_from ? 0.f : e;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pv[2 * k], pv[2 * k + 1]);
+                uint32_t dv[32];
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(dp_full + st, ph, p.status, detail_base | 0x23u));
+                tc_fence_after();
                 tmem_ld32(tm + lane_base + kColDP + 64 * st + 32 * ch, dv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int u0 = 32 * ch + 2 * k;
-                    float p0 = fast_exp2(__uint_as_float(sv[2 * k]) * c2 - lse2);
-                    float p1 = fast_exp2(__uint_as_float(sv[2 * k + 1]) * c2 - lse2);
-                    if (u0 >= mask_from) p0 = 0.f;
-                    if (u0 + 1 >= mask_from) p1 = 0.f;
-                    const float d0 = p0 * (__uint_as_float(dv[2 * k]) - dlt);
-                    const float d1 = p1 * (__uint_as_float(dv[2 * k + 1]) - dlt);
-                    pk[k] = pack_bf16x2(p0, p1);
-                    dk[k] = pack_bf16x2(d0, d1);
-                }
+                for (int k = 0; k < 16; ++k)
+                    dk[k] = pack_bf16x2(pv[2 * k] * (__uint_as_float(dv[2 * k]) - dlt),
+                                        pv[2 * k + 1] * (__uint_as_float(dv[2 * k + 1]) - dlt));
             }
             tc_fence_before();
             mbar_arrive(sdp_read + st);  // the MMA warp may refill this S/dP buffer
@@ -305,15 +315,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // forward. Per group g:
 //   S = Q K_g^T, dP = dO V_g^T        tcgen05 SS, M = 128 rows, N = 128 keys, fp32 in TMEM
 //   dS = P (dP - Delta), P = exp(scale S - LSE)   (elementwise warps, written as bf16 over the
-//                                      S columns already read: keys 0-63 into columns 0-31,
-//                                      keys 64-127 into columns 64-95)
+//                                      S columns already read: keys 32 c .. 32 c + 31 into
+//                                      columns 32 c .. 32 c + 15)
 //   dQ += dS K_g                       tcgen05 with A = dS from TMEM, B = K_g (MN-major)
 // dQ = scale dQ at the end. S is double-buffered in TMEM (S 2 x 128, dP 128, dQ 128 columns), so
 // group g+1's S and dP are formed while group g's dS is computed and used; the K ring has three
 // stages (K is read by S(g) and by dQ(g)), the V ring two.
-// Roles: warps 0-7 elementwise (two per row: keys 64 (w / 4) .. of each group; in the epilogue,
-// head-dim columns 64 (w / 4) ..), warp 8 producer (block list, Q and dO once, K lane 0, V
-// lane 1), warp 9 MMA issue and TMEM allocation.
+// Roles: warps 0-15 elementwise (four per row: keys 32 (w / 4) .. of each group, whose dS goes
+// into the first 16 of the 32 S columns the warp read; in the epilogue, head-dim columns
+// 32 (w / 4) ..), warp 16 producer (block list, Q and dO once, K lane 0, V lane 1), warp 17 MMA
+// issue and TMEM allocation.
 namespace {
 
 constexpr int kRD = 128;                       // head dim
@@ -334,10 +345,10 @@ constexpr uint32_t kRSmem = 1024 + kROffAux + kRAux;
 constexpr uint32_t kRColS = 0;     // S / dS of buffer s at 128 s
 constexpr uint32_t kRColDP = 256;
 constexpr uint32_t kRColDQ = 384;
-constexpr int kREwThreads = 256;
-constexpr int kRProducerWarp = 8;
-constexpr int kRMmaWarp = 9;
-constexpr int kRThreads = 320;
+constexpr int kREwThreads = 512;
+constexpr int kRProducerWarp = 16;
+constexpr int kRMmaWarp = 17;
+constexpr int kRThreads = 576;
 static_assert(kRSmem <= 232448, "shared memory budget");
 static_assert(kRSmem < (1 << 18), "descriptor start addresses below 2^18");
 
@@ -357,8 +368,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
     uint64_t* v_full = k_empty + kRNstK;       // NstV
     uint64_t* v_empty = v_full + kRNstV;       // NstV  dP MMAs of the group done
     uint64_t* sdp_full = v_empty + kRNstV;     // 1     S and dP of the group in TMEM
-    uint64_t* dp_read = sdp_full + 1;          // 1     elementwise warps read S and dP (256 arrivals)
-    uint64_t* ds_ready = dp_read + 1;          // 2     dS of S buffer s in TMEM (256 arrivals)
+    uint64_t* dp_read = sdp_full + 1;          // 1     elementwise warps read S and dP (512 arrivals)
+    uint64_t* ds_ready = dp_read + 1;          // 2     dS of S buffer s in TMEM (512 arrivals)
     uint64_t* dq_done = ds_ready + 2;          // 1     dQ MMAs of the group done
     uint64_t* mma_final = dq_done + 1;         // 1     teardown: every MMA issued has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
@@ -467,39 +478,30 @@ __global__ void __launch_bounds__(kRThreads, 1)
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kRD, 0, 1);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
             auto ncols_of = [&](int g) { return min(2, nsel - 2 * g) * kRB; };
-            // dP(g) = dO V_g^T into the dP columns (after the elementwise warps read dP(g-1))
-            auto issue_dp = [&](int g) -> bool {
-                const int st = g % kRNstV;
-                if (!mbar_wait(v_full + st, (g / kRNstV) & 1, p.status, detail_base | 0x11u)) return false;
+            // dP(g) = dO V_g^T into the dP columns (after the elementwise warps read dP(g-1)) and
+            // S(g) = Q K_g^T into S buffer g % 2 (after dQ(g-2) read the dS it held); the two chains
+            // alternate so the tensor pipe runs them at its independent-MMA rate
+            auto issue_sdp = [&](int g) -> bool {
+                const int sv = g % kRNstV, sk = g % kRNstK;
+                if (!mbar_wait(v_full + sv, (g / kRNstV) & 1, p.status, detail_base | 0x11u)) return false;
                 if (g > 0 && !mbar_wait(dp_read, (g - 1) & 1, p.status, detail_base | 0x12u)) return false;
-                tc_fence_after();
-                const uint32_t id = idesc_bf16_f32(128, ncols_of(g), 0, 0);
-#pragma unroll
-                for (int ks = 0; ks < kRD / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
-                    mma_bf16_ss(tm + kRColDP, smem_desc_sw128(sO + off, 16, 1024),
-                                smem_desc_sw128(sV + st * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(v_empty + st);
-                return true;
-            };
-            // S(g) = Q K_g^T into S buffer g % 2 (after dQ(g-2) read the dS it held)
-            auto issue_s = [&](int g) -> bool {
-                const int st = g % kRNstK;
-                if (!mbar_wait(k_full + st, (g / kRNstK) & 1, p.status, detail_base | 0x13u)) return false;
+                if (!mbar_wait(k_full + sk, (g / kRNstK) & 1, p.status, detail_base | 0x13u)) return false;
                 if (g > 1 && !mbar_wait(dq_done, (g - 2) & 1, p.status, detail_base | 0x14u)) return false;
                 tc_fence_after();
                 const uint32_t id = idesc_bf16_f32(128, ncols_of(g), 0, 0);
 #pragma unroll
                 for (int ks = 0; ks < kRD / 16; ++ks) {
                     const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
+                    mma_bf16_ss(tm + kRColDP, smem_desc_sw128(sO + off, 16, 1024),
+                                smem_desc_sw128(sV + sv * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
                     mma_bf16_ss(tm + kRColS + 128 * (g % 2), smem_desc_sw128(sQ + off, 16, 1024),
-                                smem_desc_sw128(sK + st * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
+                                smem_desc_sw128(sK + sk * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
                 }
+                mma_commit(v_empty + sv);
                 mma_commit(sdp_full);
                 return true;
             };
-            // dQ += dS(g) K_g (dS in TMEM: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
+            // dQ += dS(g) K_g (dS in TMEM: keys 32 c .. 32 c + 31 in columns 32 c .. 32 c + 15)
             auto issue_dq = [&](int g) -> bool {
                 const int st = g % kRNstK;
                 if (!mbar_wait(ds_ready + g % 2, (g / 2) & 1, p.status, detail_base | 0x15u)) return false;
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     if (ks < nks) {
-                        const uint32_t acol = ks < 4 ? ks * 8 : 64 + (ks - 4) * 8;
+                        const uint32_t acol = (ks / 2) * 32 + (ks % 2) * 8;
                         const uint32_t boff = static_cast<uint32_t>((ks * 16 * 128) >> 4);
                         mma_bf16_ts(tm + kRColDQ, a_tmem + acol, b0 + boff, idesc_dq, (g > 0 || ks > 0) ? 1u : 0u);
                     }
@@ -521,17 +523,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
             };
             // dP(g+1) and S(g+1) go ahead of dQ(g), so the tensor pipe forms the next group's
             // scores while the elementwise warps work on this one
-            if (ok) ok = issue_dp(0) && issue_s(0);
+            if (ok) ok = issue_sdp(0);
             for (int g = 0; ok && g < ngroups; ++g) {
-                if (g + 1 < ngroups && !(ok = issue_dp(g + 1) && issue_s(g + 1))) break;
+                if (g + 1 < ngroups && !(ok = issue_sdp(g + 1))) break;
                 ok = issue_dq(g);
             }
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- elementwise warps
-        const int q = warp % 4, ch = warp / 4;  // TMEM lane quadrant; keys 64 ch .. of each group
-        const int r = q * 32 + lane;            // row of the tile
+        const int q = warp % 4, c4 = warp / 4;  // TMEM lane quadrant; keys 32 c4 .. of each group
+        const int r = q * 32 + lane;             // row of the tile
         const bool valid = r < gh * kRB;
         const int hh = valid ? r / kRB : 0, t = r % kRB;
         const int64_t grow = (static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N + static_cast<int64_t>(i) * kRB + t;
@@ -542,25 +544,22 @@ __global__ void __launch_bounds__(kRThreads, 1)
         bool ok = true;
         for (int g = 0; g < ngroups; ++g) {
             const int ncols = min(2, nsel - 2 * g) * kRB;
-            const bool mine = ch * 64 < ncols;  // this half of the group holds keys
+            const bool mine = c4 * 32 < ncols;  // this quarter of the group holds keys
             // first column of the diagonal block in this group (128: not here)
             const int diag_lo = (diag_pos >= 0 && diag_pos / 2 == g) ? (diag_pos % 2) * kRB : 128;
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sdp_full, g & 1, p.status, detail_base | 0x20u));
             tc_fence_after();
-            const uint32_t s_col = tm + lane_base + kRColS + 128 * (g % 2) + 64 * ch;
-            uint32_t pk[32];
+            const uint32_t s_col = tm + lane_base + kRColS + 128 * (g % 2) + 32 * c4;
             if (mine) {
-                uint32_t sv[64], dv[64];
-                tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                tmem_ld32(tm + lane_base + kRColDP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(dv));
-                tmem_ld32(tm + lane_base + kRColDP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+                uint32_t sv[32], dv[32], pk[16];
+                tmem_ld32(s_col, sv);
+                tmem_ld32(tm + lane_base + kRColDP + 32 * c4, dv);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(dp_read);  // the dP columns may be overwritten
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int c0 = ch * 64 + 2 * k;  // key column in the group
+                for (int k = 0; k < 16; ++k) {
+                    const int c0 = c4 * 32 + 2 * k;  // key column in the group
                     const bool m0 = !valid || (c0 >= diag_lo && c0 - diag_lo > t);
                     const bool m1 = !valid || (c0 + 1 >= diag_lo && c0 + 1 - diag_lo > t);
                     const float p0 = fast_exp2(__uint_as_float(sv[2 * k]) * c2 - lse2);
@@ -569,8 +568,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     const float d1 = m1 ? 0.f : p1 * (__uint_as_float(dv[2 * k + 1]) - dlt);
                     pk[k] = pack_bf16x2(d0, d1);
                 }
-                tmem_st16(s_col, *reinterpret_cast<uint32_t(*)[16]>(pk));
-                tmem_st16(s_col + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+                tmem_st16(s_col, pk);
                 tmem_wait_st();
             } else {
                 mbar_arrive(dp_read);
@@ -585,26 +583,23 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tc_fence_after();
         if (ok && valid) {
             const float sc = p.scale;
-            uint4* dst = reinterpret_cast<uint4*>(p.dQ + grow * kRD + ch * 64);
+            uint4* dst = reinterpret_cast<uint4*>(p.dQ + grow * kRD + c4 * 32);
+            uint32_t o[32];
+            if (ngroups > 0) {
+                tmem_ld32(tm + lane_base + kRColDQ + c4 * 32, o);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t o[32];
-                if (ngroups > 0) {
-                    tmem_ld32(tm + lane_base + kRColDQ + ch * 64 + c * 32, o);
-                    tmem_wait_ld();
-                } else {
+                for (int x = 0; x < 32; ++x) o[x] = 0u;
+            }
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) o[x] = 0u;
-                }
+            for (int k = 0; k < 4; ++k) {
+                uint32_t v[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint32_t v[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        v[e] = pack_bf16x2(__uint_as_float(o[8 * k + 2 * e]) * sc,
-                                           __uint_as_float(o[8 * k + 2 * e + 1]) * sc);
-                    dst[c * 4 + k] = make_uint4(v[0], v[1], v[2], v[3]);
-                }
+                for (int e = 0; e < 4; ++e)
+                    v[e] = pack_bf16x2(__uint_as_float(o[8 * k + 2 * e]) * sc,
+                                       __uint_as_float(o[8 * k + 2 * e + 1]) * sc);
+                dst[k] = make_uint4(v[0], v[1], v[2], v[3]);
             }
         }
     }
