@@ -42,6 +42,12 @@ constexpr uint32_t kKSub = kTB * 128;           // [64 keys x 128 B] tile
 constexpr uint32_t kKVBytes = kDS * kKSub;      // K_j or V_j
 constexpr uint32_t kQOBytes = kDS * kSub;       // the Q or the dO rows of one tile
 constexpr uint32_t kPDBytes = 128 * 128;        // P or dS of one tile: [128 rows x 64 keys] bf16
+// A descriptor moved by `bytes` (a multiple of 16): the start-address field holds address / 16
+// in 14 bits and shared memory ends below 2^18 bytes, so the add never carries out of it. The
+// MMA lane forms each operand's descriptor once and only adds offsets, which keeps its
+// instruction count per MMA small beside the busy elementwise warps on its sub-partition.
+__device__ __forceinline__ uint64_t dmove(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 constexpr int kNst = 2;
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kKVBytes;
@@ -149,7 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && ntiles > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTB, 0, 0);  // S, dP: A and B K-major
             constexpr uint32_t idesc_g = idesc_bf16_f32(128, kTB, 1, 1);  // dV^T, dK^T: A and B MN-major
-            const uint32_t sK = smem_u32(base + kOffK), sV = smem_u32(base + kOffV);
+            const uint32_t s0 = smem_u32(base);
+            const uint64_t dK = smem_desc_sw128(s0 + kOffK, 16, 1024), dV = smem_desc_sw128(s0 + kOffV, 16, 1024);
+            const uint64_t dQk = smem_desc_sw128(s0 + kOffQ, 16, 1024);         // Q / dO, K-major
+            const uint64_t dQm = smem_desc_sw128(s0 + kOffQ, kSub, 1024);       // Q / dO, MN-major
+            const uint64_t dPm = smem_desc_sw128(s0 + kOffP, kPDBytes, 1024);   // P / dS, MN-major
             bool ok = mbar_wait(kv_full, 0, p.status, detail_base | 0x10u);
             for (int r0 = 0; ok && r0 < ntiles; r0 += kNst) {
                 const int r1 = min(r0 + kNst, ntiles);
@@ -159,19 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = mbar_wait(qo_full + st, ph, p.status, detail_base | 0x11u))) break;
                     if (!(ok = mbar_wait(sdp_read + st, ph ^ 1, p.status, detail_base | 0x12u))) break;
                     tc_fence_after();
-                    const uint32_t sQ = smem_u32(base + kOffQ + st * 2 * kQOBytes), sO = sQ + kQOBytes;
+                    const uint64_t dq = dmove(dQk, st * 2 * kQOBytes), dout = dmove(dq, kQOBytes);
 #pragma unroll
                     for (int ks = 0; ks < kTD / 16; ++ks) {
                         const uint32_t oa = (ks / 4) * kSub + (ks % 4) * 32, ob = (ks / 4) * kKSub + (ks % 4) * 32;
-                        mma_bf16_ss(tm + kColS + 64 * st, smem_desc_sw128(sQ + oa, 16, 1024),
-                                    smem_desc_sw128(sK + ob, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                        mma_bf16_ss(tm + kColS + 64 * st, dmove(dq, oa), dmove(dK, ob), idesc_s, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(s_full + st);  // the exponentials start while dP is formed
 #pragma unroll
                     for (int ks = 0; ks < kTD / 16; ++ks) {
                         const uint32_t oa = (ks / 4) * kSub + (ks % 4) * 32, ob = (ks / 4) * kKSub + (ks % 4) * 32;
-                        mma_bf16_ss(tm + kColDP + 64 * st, smem_desc_sw128(sO + oa, 16, 1024),
-                                    smem_desc_sw128(sV + ob, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                        mma_bf16_ss(tm + kColDP + 64 * st, dmove(dout, oa), dmove(dV, ob), idesc_s, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(dp_full + st);
                 }
@@ -181,19 +189,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int su = u % kNst;
                     if (!(ok = mbar_wait(p_ready + su, (u / kNst) & 1, p.status, detail_base | 0x13u))) break;
                     tc_fence_after();
-                    const uint32_t sQ = smem_u32(base + kOffQ + su * 2 * kQOBytes), sO = sQ + kQOBytes;
-                    const uint32_t sP = smem_u32(base + kOffP + su * 2 * kPDBytes), sdS = sP + kPDBytes;
+                    const uint64_t dq = dmove(dQm, su * 2 * kQOBytes), dout = dmove(dq, kQOBytes);
+                    const uint64_t dp = dmove(dPm, su * 2 * kPDBytes), dds = dmove(dp, kPDBytes);
 #pragma unroll
                     for (int ks = 0; ks < 128 / 16; ++ks) {
                         const uint32_t ro = ks * 16 * 128;
-                        mma_bf16_ss(tm + kColDV, smem_desc_sw128(sO + ro, kSub, 1024),
-                                    smem_desc_sw128(sP + ro, kPDBytes, 1024), idesc_g, (u > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(tm + kColDV, dmove(dout, ro), dmove(dp, ro), idesc_g, (u > 0 || ks > 0) ? 1u : 0u);
                     }
 #pragma unroll
                     for (int ks = 0; ks < 128 / 16; ++ks) {
                         const uint32_t ro = ks * 16 * 128;
-                        mma_bf16_ss(tm + kColDK, smem_desc_sw128(sQ + ro, kSub, 1024),
-                                    smem_desc_sw128(sdS + ro, kPDBytes, 1024), idesc_g, (u > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(tm + kColDK, dmove(dq, ro), dmove(dds, ro), idesc_g, (u > 0 || ks > 0) ? 1u : 0u);
                     }
                     mma_commit(qo_empty + su);
                 }
@@ -473,8 +479,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
         __syncwarp();
     } else if (warp == kRMmaWarp) {
         if (lane == 0 && ngroups > 0) {
-            const uint32_t sQ = smem_u32(base + kROffQ), sO = smem_u32(base + kROffO);
-            const uint32_t sK = smem_u32(base + kROffK), sV = smem_u32(base + kROffV);
+            const uint32_t s0 = smem_u32(base);
+            const uint64_t dQk = smem_desc_sw128(s0 + kROffQ, 16, 1024), dOk = smem_desc_sw128(s0 + kROffO, 16, 1024);
+            const uint64_t dKk = smem_desc_sw128(s0 + kROffK, 16, 1024), dVk = smem_desc_sw128(s0 + kROffV, 16, 1024);
+            const uint64_t dKm = smem_desc_sw128(s0 + kROffK, kRSub, 1024);  // K as the MN-major B of dS.K
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kRD, 0, 1);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
             auto ncols_of = [&](int g) { return min(2, nsel - 2 * g) * kRB; };
@@ -489,13 +497,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 if (g > 1 && !mbar_wait(dq_done, (g - 2) & 1, p.status, detail_base | 0x14u)) return false;
                 tc_fence_after();
                 const uint32_t id = idesc_bf16_f32(128, ncols_of(g), 0, 0);
+                const uint64_t dv = dmove(dVk, sv * kRTile), dk = dmove(dKk, sk * kRTile);
+                const uint32_t s_col = tm + kRColS + 128 * (g % 2);
 #pragma unroll
                 for (int ks = 0; ks < kRD / 16; ++ks) {
                     const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
-                    mma_bf16_ss(tm + kRColDP, smem_desc_sw128(sO + off, 16, 1024),
-                                smem_desc_sw128(sV + sv * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
-                    mma_bf16_ss(tm + kRColS + 128 * (g % 2), smem_desc_sw128(sQ + off, 16, 1024),
-                                smem_desc_sw128(sK + sk * kRTile + off, 16, 1024), id, ks > 0 ? 1u : 0u);
+                    mma_bf16_ss(tm + kRColDP, dmove(dOk, off), dmove(dv, off), id, ks > 0 ? 1u : 0u);
+                    mma_bf16_ss(s_col, dmove(dQk, off), dmove(dk, off), id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(v_empty + sv);
                 mma_commit(sdp_full);
@@ -508,7 +516,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 tc_fence_after();
                 const int nks = ncols_of(g) / 16;
                 const uint32_t a_tmem = tm + kRColS + 128 * (g % 2);
-                const uint64_t b0 = smem_desc_sw128(sK + st * kRTile, kRSub, 1024);
+                const uint64_t b0 = dmove(dKm, st * kRTile);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     if (ks < nks) {
