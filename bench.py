@@ -251,7 +251,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = rank_workload(bench_workload(args), rank)
-    shape = pisa.Shape.of(w)
+    shape = pisa.Shape.of(w, select_per_qhead=int(args.per_qhead))
     q, k, v = (workloads.device_tensor(w, t, dev) for t in ("q", "k", "v"))
     ws = pisa.new_workspace(shape, dev)
     pyr = torch.empty(pisa.pyramid_size(shape) // 4, dtype=torch.float32, device=dev)
@@ -346,13 +346,18 @@ def run_gpu(args, world, rank, local):
 
     if rank != 0:
         return
-    cpu = oracle_sample(bench_workload(args)) if world == 1 and not args.no_cpu_baseline else None
-    traffic = profiled_traffic("attn_prefill_gqa128k.md", ATTN_SOURCES)
+    cpu = (oracle_sample(bench_workload(args))
+           if world == 1 and not args.no_cpu_baseline and not args.per_qhead else None)
+    # the recorded ncu traffic belongs to the group-shared launch (two 128-row tiles per CTA)
+    traffic = None if args.per_qhead else profiled_traffic("attn_prefill_gqa128k.md", ATTN_SOURCES)
+    config = config_dict(w, world)
+    if args.per_qhead:
+        config["workload"] += ", per-query-head selection"
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC + (" [per-query-head selection]" if args.per_qhead else ""), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy, bf16 RNE)",
-        "config": config_dict(w, world),
+        "config": config,
         "effective_tflops": attn_flops * world / (ms_step / 1e3) / 1e12,
         "fused_roofline_frac": roof_s / (ms_step / 1e3),
         "stages_ms": {"pyramid": stage_ms[0], "select": stage_ms[1], "attention": stage_ms[2]},
@@ -361,7 +366,8 @@ def run_gpu(args, world, rank, local):
             "select_gbs_qread": sel_bytes / (stage_ms[1] / 1e3) / 1e9,
             "attention_tflops": achieved,
         },
-        "roofline": {"bound": "tensor", "kernel": "attn_prefill_kernel<128,64,2>", "achieved": achieved,
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_prefill_kernel<128,64,%d>" % (1 if args.per_qhead else 2), "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                      "peak_source": f"{how} bf16 dense (burst)", "traffic": traffic,
                      "flops_per_launch": attn_flops},
@@ -555,6 +561,8 @@ def main():
                     help="prefill workload to time (default: the N=128K GQA workload)")
     ap.add_argument("--seq", type=int, default=0, help="override the sequence length (smaller profiling cases)")
     ap.add_argument("--backward", action="store_true", help="time the backward step instead of the forward")
+    ap.add_argument("--per-qhead", action="store_true",
+                    help="forward with one selection per query head (select_per_qhead = 1); no CPU baseline")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.impl == "reference":
