@@ -46,3 +46,19 @@ def assert_pyramid_close(pyr_gpu, levels_ref, offsets):
         got = pyr_gpu[offsets[l]:offsets[l] + lev.shape[0]]
         err = np.abs(got - lev)
         assert np.all(err <= PYR_TOL + PYR_TOL * np.abs(lev)), f"level {l}: max err {err.max():.3e}"
+
+
+def compact_row_problem(sel, i: int, block: int, causal: bool, t: np.ndarray):
+    """Index plumbing for checking one query block on its own: the keys of its selected blocks
+    `sel` (ascending) laid end to end, and query positions `t` (within block i) moved so that a
+    causal mask over the compacted positions hides exactly what it hid in the full plane: every
+    key of a block j < i stays visible, and in the diagonal block (j = i, which sorts last) key u
+    is visible from query t >= u. Returns (key rows in the full plane, compacted query positions,
+    compacted block ids)."""
+    n = len(sel)
+    key_rows = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel]) if n else np.zeros(0, int)
+    if causal and n and sel[-1] == i:
+        q_pos = (n - 1) * block + t
+    else:
+        q_pos = n * block + t
+    return key_rows, q_pos, list(range(n))

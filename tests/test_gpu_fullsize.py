@@ -109,3 +109,71 @@ def test_decode128k(cuda_device):
     w = workloads.WORKLOADS["decode128k"]
     shape, pyr, idx, o, lse = _run(w, cuda_device)
     _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (17, 3), (63, 7)], 1, 1, 4)
+
+
+def test_gqa128k_backward_sampled(cuda_device):
+    """The backward at the bench's full size (128K GQA, `bench.py --backward`): dQ of sampled query
+    blocks and dK, dV of sampled key blocks (one with a list of ~90 query blocks x 4 heads, i.e.
+    ~180 column-pass tiles) against the fp64 oracle, each part computed on its own from the rows
+    and keys it depends on."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = workloads.WORKLOADS["gqa128k"]
+    shape = pisa.Shape.of(w)
+    q, k, v = (workloads.device_tensor(w, t, cuda_device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    gen = torch.Generator(device="cpu").manual_seed(w.seed + 1000)
+    do_h = torch.randn(tuple(q.shape), generator=gen).to(torch.bfloat16)
+    do = do_h.to(cuda_device)
+    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, "backward")
+    del o, lse, q, k, v
+    idx_h = idx.cpu().numpy()
+    B, g, blk, nqb = 0, w.group, w.block, shape.n_qblocks
+    scale = 1.0 / math.sqrt(w.head_dim)
+    t = np.arange(blk)
+    rel_max, rel_mean = 2e-2, 1e-3
+
+    def close(got, ref, what):
+        err = np.abs(got - ref)
+        top = np.abs(ref).max()
+        assert err.max() <= rel_max * top, f"{what}: max err {err.max():.3e} vs max |ref| {top:.3e}"
+        assert err.mean() <= rel_mean * top, f"{what}: mean err {err.mean():.3e} vs max |ref| {top:.3e}"
+
+    for kvh in (0, 5):
+        K = workloads.plane_f32(w, "k", B, kvh)
+        V = workloads.plane_f32(w, "v", B, kvh)
+        heads = list(range(kvh * g, (kvh + 1) * g))
+        Qh = {h: workloads.plane_f32(w, "q", B, h) for h in heads}
+        dOh = {h: do_h[B, h].float().numpy() for h in heads}
+
+        def row_grads(i, h):
+            sel = [int(j) for j in idx_h[B, kvh, i] if j >= 0]
+            rows, q_pos, blocks = gu.compact_row_problem(sel, i, blk, True, t)
+            qr = slice(i * blk, (i + 1) * blk)
+            dq_r, dk_r, dv_r = oracle.attend_backward(Qh[h][qr], q_pos, K[rows], V[rows], blocks, blk, True,
+                                                      scale, dOh[h][qr])
+            return sel, dq_r, dk_r, dv_r
+
+        # dQ of sampled query blocks (first, last, a needle target, random)
+        rng = np.random.Generator(np.random.PCG64(40 + kvh))
+        target = workloads.needles(w, B, kvh)[0][0]
+        for i in sorted({0, nqb - 1, target} | set(rng.choice(nqb, size=3, replace=False).tolist())):
+            for h in heads:
+                _, dq_r, _, _ = row_grads(i, h)
+                close(gu.host_f32(dq[B, h, i * blk:(i + 1) * blk]), dq_r, f"dQ kvh{kvh} h{h} i{i}")
+        # dK, dV of sampled key blocks: sum over every (query block, head) whose selection holds it
+        for j in ((nqb // 4 + 3, nqb - 1) if kvh == 0 else (nqb // 2 + 7, nqb - 1)):
+            users = [i for i in range(j, nqb) if j in idx_h[B, kvh, i]]
+            dk_ref = np.zeros((blk, w.head_dim))
+            dv_ref = np.zeros((blk, w.head_dim))
+            for i in users:
+                for h in heads:
+                    sel, _, dk_r, dv_r = row_grads(i, h)
+                    m = sel.index(j)
+                    dk_ref += dk_r[m * blk:(m + 1) * blk]
+                    dv_ref += dv_r[m * blk:(m + 1) * blk]
+            close(gu.host_f32(dk[B, kvh, j * blk:(j + 1) * blk]), dk_ref, f"dK kvh{kvh} j{j} ({len(users)} users)")
+            close(gu.host_f32(dv[B, kvh, j * blk:(j + 1) * blk]), dv_ref, f"dV kvh{kvh} j{j} ({len(users)} users)")
