@@ -14,13 +14,16 @@
 // 4. At each level every candidate gets an fp32 dot product with the query
 //    summary (eight lanes per candidate, so each warp load covers four whole
 //    128-byte lines of node vectors; a three-step shuffle adds the lanes). Candidates are ranked by
-//    a 64-bit key (order-preserving score bits, then inverted node index), so
-//    that a bitonic sort in shared memory orders by higher score and, on equal
-//    scores, lower index. The kept nodes' eligible children become the next
-//    candidates; holes (ineligible children) carry key 0 and sort last.
+//    a 64-bit key (order-preserving score bits, then inverted node index): higher score first
+//    and, on equal scores, lower index. The K_l-th largest key is found by bisection with
+//    CTA-wide counts (the score word first, the index word only when scores tie at the cut),
+//    and the kept candidates are compacted in candidate order. Candidates are produced in
+//    ascending node order at every level (the first scored level's eligible nodes, then the
+//    children of the kept parents, parents ascending), so every kept list is ascending; holes
+//    (ineligible children) carry key 0 and are never kept.
 // 5. The kept level-0 blocks are written in ascending order, padded with -1.
 //    Forced blocks (sink, local) are left out of the level-0 candidates, which
-//    then keep K minus their count, and join the output before the final sort.
+//    then keep K minus their count, and are merged into the ascending output.
 #include <cuda_bf16.h>
 
 #include "pisa_device.cuh"
@@ -49,44 +52,25 @@ __device__ __forceinline__ int32_t key_node(uint64_t k) {
     return static_cast<int32_t>(~static_cast<uint32_t>(k & 0xFFFFFFFFull));
 }
 
-// Sorts keys[0, n) in descending order; n is a power of two.
-__device__ void bitonic_desc(uint64_t* keys, int n) {
-    for (int k = 2; k <= n; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int t = threadIdx.x; t < n; t += kSelThreads) {
-                const int u = t ^ j;
-                if (u > t) {
-                    const uint64_t a = keys[t], b = keys[u];
-                    const bool desc = (t & k) == 0;
-                    if (desc ? (a < b) : (a > b)) {
-                        keys[t] = b;
-                        keys[u] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
+// CTA-wide sum (or max) of one value per thread, one barrier per call: the four warps' partial
+// results go to one of two slot sets, alternated by `phase`, so a slot set is rewritten only
+// after the barrier of the next call, which every thread reaches after reading it.
+__device__ __forceinline__ int cta_sum(int v, int* slots, int& phase) {
+    v = __reduce_add_sync(0xFFFFFFFFu, v);
+    int* b = slots + 4 * (phase & 1);
+    if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
+    __syncthreads();
+    ++phase;
+    return b[0] + b[1] + b[2] + b[3];
 }
 
-// Sorts ints[0, n) ascending; n is a power of two.
-__device__ void bitonic_asc(int32_t* v, int n) {
-    for (int k = 2; k <= n; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int t = threadIdx.x; t < n; t += kSelThreads) {
-                const int u = t ^ j;
-                if (u > t) {
-                    const int32_t a = v[t], b = v[u];
-                    const bool asc = (t & k) == 0;
-                    if (asc ? (a > b) : (a < b)) {
-                        v[t] = b;
-                        v[u] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
+__device__ __forceinline__ uint32_t cta_max(uint32_t v, int* slots, int& phase) {
+    v = __reduce_max_sync(0xFFFFFFFFu, v);
+    uint32_t* b = reinterpret_cast<uint32_t*>(slots + 4 * (phase & 1));
+    if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
+    __syncthreads();
+    ++phase;
+    return max(max(b[0], b[1]), max(b[2], b[3]));
 }
 
 __device__ __forceinline__ int next_pow2(int n) {
@@ -100,10 +84,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     extern __shared__ __align__(16) uint8_t sm[];
     uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                         // [cap]
     int32_t* cand = reinterpret_cast<int32_t*>(keys + cap);                    // [cap]
-    float* qs = reinterpret_cast<float*>(cand + cap);                          // [D]
+    int32_t* kept = cand + cap;                                                // [cap]
+    float* qs = reinterpret_cast<float*>(kept + cap);                          // [D]
     float* part = qs + D;                                                      // [L][D]
     __shared__ int s_nvalid;
     __shared__ float s_margin;
+    __shared__ int s_slots[8];  // CTA reductions (two alternating sets of four warp partials)
+    __shared__ int s_scan[4];   // warp totals of the compaction scan
 
     const int i = blockIdx.x, hs = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x;
@@ -125,7 +112,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 ch[u] = u < nch ? plane[(p.loff[l - 1] + c_l * p.factor + u) * D + d] : 0.f;
-            for (int u = 8; u < nch; ++u) sum += static_cast<float>(wb) * plane[(p.loff[l - 1] + c_l * p.factor + u) * D + d];
+            for (int u = 8; u < nch; ++u)
+                sum += static_cast<float>(wb) * plane[(p.loff[l - 1] + c_l * p.factor + u) * D + d];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 if (u < nch) sum += static_cast<float>(wb) * ch[u];
@@ -148,22 +136,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             break;
         }
     }
-    int nkeep;
-    int32_t* out_ids = cand;  // reused for the final ascending sort
     int32_t f0, f1;
     const int nf = forced_blocks(p.forced, p.decode ? p.n0_valid - 1 : i, p.budget[0], f0, f1);
+    int32_t* dst = p.idx + row * p.topk;
+    const int warp = tid >> 5, lane = tid & 31;
+    int phase = 0;
     if (l0 < 0) {
-        nkeep = last + 1;  // every eligible block fits the budget
-        const int n = next_pow2(nkeep);
-        for (int t = tid; t < n; t += kSelThreads) out_ids[t] = t < nkeep ? t : 0x7FFFFFFF;
-        __syncthreads();
+        // every eligible block fits the budget (the forced ones among them)
+        const int nkeep = last + 1;
+        for (int t = tid; t < p.topk; t += kSelThreads) dst[t] = t < nkeep ? t : -1;
     } else {
         int ncand = static_cast<int>(last / p.width[l0] + 1);
         // at level 0 the forced blocks (all eligible) are not candidates
         for (int t = tid; t < ncand; t += kSelThreads) cand[t] = (l0 == 0 && (t == f0 || t == f1)) ? -1 : t;
         if (tid == 0) s_nvalid = l0 == 0 ? ncand - nf : ncand;
         __syncthreads();
-        nkeep = 0;
         for (int l = l0; l >= 0; --l) {
             const int n = next_pow2(ncand);
             const int64_t c_part = last / p.width[l];
@@ -206,46 +193,118 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             }
             __syncthreads();
             const int nvalid = s_nvalid;
-            bitonic_desc(keys, n);
             const int k_l = l == 0 ? p.budget[0] - nf : p.budget[l];
-            nkeep = min(k_l, nvalid);
-            if (tid == 0 && nvalid > k_l && k_l > 0) {
-                const float a = order_bits_inv(static_cast<uint32_t>(keys[k_l - 1] >> 32));
-                const float c = order_bits_inv(static_cast<uint32_t>(keys[k_l] >> 32));
-                const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
-                s_margin = fminf(s_margin, rel);
+            // this thread's candidates form one contiguous run, so the compaction keeps their order
+            const int per = (ncand + kSelThreads - 1) / kSelThreads;
+            const int s0 = min(ncand, tid * per), s1 = min(ncand, s0 + per);
+            // kept: key >= (th_hi, th_lo) as (score word, index word); (0, 1) keeps every valid key
+            // (a valid key's score word is never 0; a hole's key is 0)
+            uint32_t th_hi = 0, th_lo = 1;
+            if (nvalid > k_l && k_l <= 0) {
+                th_hi = 0xFFFFFFFFu;  // nothing is kept (finite scores never reach this word)
+                th_lo = 0xFFFFFFFFu;
+            } else if (nvalid > k_l) {
+                // score word of the K_l-th largest key: the largest h with at least K_l words >= h
+                th_hi = 0;
+                for (int bit = 31; bit >= 0; --bit) {
+                    const uint32_t c = th_hi | (1u << bit);
+                    int cnt = 0;
+                    for (int t = s0; t < s1; ++t) cnt += static_cast<uint32_t>(keys[t] >> 32) >= c;
+                    if (cta_sum(cnt, s_slots, phase) >= k_l) th_hi = c;
+                }
+                int gt = 0, eq = 0;
+                uint32_t below = 0;  // largest score word under th_hi: the (K_l+1)-th score if no tie
+                for (int t = s0; t < s1; ++t) {
+                    const uint32_t h = static_cast<uint32_t>(keys[t] >> 32);
+                    gt += h > th_hi;
+                    eq += h == th_hi;
+                    if (h < th_hi) below = max(below, h);
+                }
+                gt = cta_sum(gt, s_slots, phase);
+                eq = cta_sum(eq, s_slots, phase);
+                below = cta_max(below, s_slots, phase);
+                const int need = k_l - gt;  // kept among the keys whose score word is th_hi
+                th_lo = 0;
+                if (eq > need) {
+                    // equal scores at the cut: the `need` largest index words (lower nodes) among them
+                    for (int bit = 31; bit >= 0; --bit) {
+                        const uint32_t c = th_lo | (1u << bit);
+                        int cnt = 0;
+                        for (int t = s0; t < s1; ++t) {
+                            const uint64_t key = keys[t];
+                            cnt += static_cast<uint32_t>(key >> 32) == th_hi && static_cast<uint32_t>(key) >= c;
+                        }
+                        if (cta_sum(cnt, s_slots, phase) >= need) th_lo = c;
+                    }
+                    below = th_hi;  // the (K_l+1)-th score equals the K_l-th
+                }
+                if (tid == 0) {
+                    const float a = order_bits_inv(th_hi);
+                    const float c = order_bits_inv(below);
+                    const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
+                    s_margin = fminf(s_margin, rel);
+                }
             }
+            const uint64_t th = (static_cast<uint64_t>(th_hi) << 32) | th_lo;
+            // stable compaction of the kept candidates
+            int mine = 0;
+            for (int t = s0; t < s1; ++t) mine += keys[t] >= th;
+            int incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) s_scan[warp] = incl;
+            __syncthreads();
+            int pos = incl - mine;
+            for (int w = 0; w < warp; ++w) pos += s_scan[w];
+            const int nkeep = s_scan[0] + s_scan[1] + s_scan[2] + s_scan[3];
+            for (int t = s0; t < s1; ++t)
+                if (keys[t] >= th) kept[pos++] = cand[t];
+            __syncthreads();  // kept[] complete; s_nvalid and s_scan read by every thread
             if (l > 0) {
+                // the next candidates: children of the kept parents, parents ascending
                 const int64_t last_below = last / p.width[l - 1];
                 const int n_below = p.lsize[l - 1];
                 const int slots = nkeep * p.factor;
-                __syncthreads();  // every thread has read s_nvalid
                 if (tid == 0) s_nvalid = 0;
                 __syncthreads();
-                int mine = 0;
+                int valid_here = 0;
                 for (int t = tid; t < slots; t += kSelThreads) {
-                    const int32_t c = key_node(keys[t / p.factor]);
+                    const int32_t c = kept[t / p.factor];
                     const int64_t ch = static_cast<int64_t>(c) * p.factor + (t % p.factor);
                     const bool ok = ch <= last_below && ch < n_below && (l > 1 || (ch != f0 && ch != f1));
                     cand[t] = ok ? static_cast<int32_t>(ch) : -1;
-                    mine += ok;
+                    valid_here += ok;
                 }
-                if (mine) atomicAdd(&s_nvalid, mine);
+                if (valid_here) atomicAdd(&s_nvalid, valid_here);
                 ncand = slots;
                 __syncthreads();
             } else {
-                const int nn = next_pow2(nkeep + nf);
-                __syncthreads();
-                for (int t = tid; t < nn; t += kSelThreads)
-                    out_ids[t] = t < nkeep ? key_node(keys[t]) : t < nkeep + nf ? (t == nkeep ? f0 : f1) : 0x7FFFFFFF;
-                nkeep += nf;
-                __syncthreads();
+                // the ascending kept blocks with the forced ones merged in, padded with -1
+                for (int t = tid; t < nkeep; t += kSelThreads) {
+                    const int32_t v = kept[t];
+                    dst[t + (f0 >= 0 && f0 < v) + (f1 >= 0 && f1 < v)] = v;
+                }
+                if (tid < 2) {
+                    const int32_t f = tid == 0 ? f0 : f1, other = tid == 0 ? f1 : f0;
+                    if (f >= 0) {
+                        int lo = 0, hi = nkeep;  // kept blocks below f
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (kept[mid] < f)
+                                lo = mid + 1;
+                            else
+                                hi = mid;
+                        }
+                        dst[lo + (other >= 0 && other < f)] = f;
+                    }
+                }
+                for (int t = nkeep + nf + tid; t < p.topk; t += kSelThreads) dst[t] = -1;
             }
         }
     }
-    bitonic_asc(out_ids, next_pow2(nkeep));
-    int32_t* dst = p.idx + row * p.topk;
-    for (int t = tid; t < p.topk; t += kSelThreads) dst[t] = t < nkeep ? out_ids[t] : -1;
     if (p.margin != nullptr && tid == 0) p.margin[row] = s_margin;
 }
 
@@ -260,7 +319,7 @@ bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_
         return launch_select_dense(p, batch, cap, st);
     }
     *launches += 1;
-    const size_t smem = static_cast<size_t>(cap) * (sizeof(uint64_t) + sizeof(int32_t)) +
+    const size_t smem = static_cast<size_t>(cap) * (sizeof(uint64_t) + 2 * sizeof(int32_t)) +
                         static_cast<size_t>(p.D) * (1 + p.L) * sizeof(float);
     dim3 grid(p.nqb, p.Hsel, batch);
     if (p.D == 64) {
