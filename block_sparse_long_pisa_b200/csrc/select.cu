@@ -15,9 +15,10 @@
 //    summary (eight lanes per candidate, so each warp load covers four whole
 //    128-byte lines of node vectors; a three-step shuffle adds the lanes). Candidates are ranked by
 //    a 64-bit key (order-preserving score bits, then inverted node index): higher score first
-//    and, on equal scores, lower index. The K_l-th largest key is found by bisection with
-//    CTA-wide counts (the score word first, the index word only when scores tie at the cut),
-//    and the kept candidates are compacted in candidate order. Candidates are produced in
+//    and, on equal scores, lower index. One warp finds the K_l-th largest key by bisection with
+//    warp-wide counts (the score word first, the index word only when scores tie at the cut;
+//    a CTA barrier per step costs several hundred cycles here) and compacts the kept
+//    candidates in candidate order. Candidates are produced in
 //    ascending node order at every level (the first scored level's eligible nodes, then the
 //    children of the kept parents, parents ascending), so every kept list is ascending; holes
 //    (ineligible children) carry key 0 and are never kept.
@@ -52,27 +53,6 @@ __device__ __forceinline__ int32_t key_node(uint64_t k) {
     return static_cast<int32_t>(~static_cast<uint32_t>(k & 0xFFFFFFFFull));
 }
 
-// CTA-wide sum (or max) of one value per thread, one barrier per call: the four warps' partial
-// results go to one of two slot sets, alternated by `phase`, so a slot set is rewritten only
-// after the barrier of the next call, which every thread reaches after reading it.
-__device__ __forceinline__ int cta_sum(int v, int* slots, int& phase) {
-    v = __reduce_add_sync(0xFFFFFFFFu, v);
-    int* b = slots + 4 * (phase & 1);
-    if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
-    __syncthreads();
-    ++phase;
-    return b[0] + b[1] + b[2] + b[3];
-}
-
-__device__ __forceinline__ uint32_t cta_max(uint32_t v, int* slots, int& phase) {
-    v = __reduce_max_sync(0xFFFFFFFFu, v);
-    uint32_t* b = reinterpret_cast<uint32_t*>(slots + 4 * (phase & 1));
-    if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
-    __syncthreads();
-    ++phase;
-    return max(max(b[0], b[1]), max(b[2], b[3]));
-}
-
 __device__ __forceinline__ int next_pow2(int n) {
     int p = 1;
     while (p < n) p <<= 1;
@@ -89,8 +69,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     float* part = qs + D;                                                      // [L][D]
     __shared__ int s_nvalid;
     __shared__ float s_margin;
-    __shared__ int s_slots[8];  // CTA reductions (two alternating sets of four warp partials)
-    __shared__ int s_scan[4];   // warp totals of the compaction scan
+    __shared__ int s_scan[1];   // kept count of the level
 
     const int i = blockIdx.x, hs = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x;
@@ -140,7 +119,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     const int nf = forced_blocks(p.forced, p.decode ? p.n0_valid - 1 : i, p.budget[0], f0, f1);
     int32_t* dst = p.idx + row * p.topk;
     const int warp = tid >> 5, lane = tid & 31;
-    int phase = 0;
     if (l0 < 0) {
         // every eligible block fits the budget (the forced ones among them)
         const int nkeep = last + 1;
@@ -194,75 +172,76 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             __syncthreads();
             const int nvalid = s_nvalid;
             const int k_l = l == 0 ? p.budget[0] - nf : p.budget[l];
-            // this thread's candidates form one contiguous run, so the compaction keeps their order
-            const int per = (ncand + kSelThreads - 1) / kSelThreads;
-            const int s0 = min(ncand, tid * per), s1 = min(ncand, s0 + per);
-            // kept: key >= (th_hi, th_lo) as (score word, index word); (0, 1) keeps every valid key
-            // (a valid key's score word is never 0; a hole's key is 0)
-            uint32_t th_hi = 0, th_lo = 1;
-            if (nvalid > k_l && k_l <= 0) {
-                th_hi = 0xFFFFFFFFu;  // nothing is kept (finite scores never reach this word)
-                th_lo = 0xFFFFFFFFu;
-            } else if (nvalid > k_l) {
-                // score word of the K_l-th largest key: the largest h with at least K_l words >= h
-                th_hi = 0;
-                for (int bit = 31; bit >= 0; --bit) {
-                    const uint32_t c = th_hi | (1u << bit);
-                    int cnt = 0;
-                    for (int t = s0; t < s1; ++t) cnt += static_cast<uint32_t>(keys[t] >> 32) >= c;
-                    if (cta_sum(cnt, s_slots, phase) >= k_l) th_hi = c;
-                }
-                int gt = 0, eq = 0;
-                uint32_t below = 0;  // largest score word under th_hi: the (K_l+1)-th score if no tie
-                for (int t = s0; t < s1; ++t) {
-                    const uint32_t h = static_cast<uint32_t>(keys[t] >> 32);
-                    gt += h > th_hi;
-                    eq += h == th_hi;
-                    if (h < th_hi) below = max(below, h);
-                }
-                gt = cta_sum(gt, s_slots, phase);
-                eq = cta_sum(eq, s_slots, phase);
-                below = cta_max(below, s_slots, phase);
-                const int need = k_l - gt;  // kept among the keys whose score word is th_hi
-                th_lo = 0;
-                if (eq > need) {
-                    // equal scores at the cut: the `need` largest index words (lower nodes) among them
+            // warp 0 selects: counts by warp reductions, no CTA barrier per bisection step
+            if (warp == 0) {
+                // this lane's candidates form one contiguous run, so the compaction keeps their order
+                const int per = (ncand + 31) / 32;
+                const int s0 = min(ncand, lane * per), s1 = min(ncand, s0 + per);
+                // kept: key >= (th_hi, th_lo) as (score word, index word); (0, 1) keeps every valid
+                // key (a valid key's score word is never 0; a hole's key is 0)
+                uint32_t th_hi = 0, th_lo = 1;
+                if (nvalid > k_l && k_l <= 0) {
+                    th_hi = 0xFFFFFFFFu;  // nothing is kept (finite scores never reach this word)
+                    th_lo = 0xFFFFFFFFu;
+                } else if (nvalid > k_l) {
+                    // score word of the K_l-th largest key: the largest h with at least K_l words >= h
+                    th_hi = 0;
                     for (int bit = 31; bit >= 0; --bit) {
-                        const uint32_t c = th_lo | (1u << bit);
+                        const uint32_t c = th_hi | (1u << bit);
                         int cnt = 0;
-                        for (int t = s0; t < s1; ++t) {
-                            const uint64_t key = keys[t];
-                            cnt += static_cast<uint32_t>(key >> 32) == th_hi && static_cast<uint32_t>(key) >= c;
-                        }
-                        if (cta_sum(cnt, s_slots, phase) >= need) th_lo = c;
+                        for (int t = s0; t < s1; ++t) cnt += static_cast<uint32_t>(keys[t] >> 32) >= c;
+                        if (static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, cnt)) >= k_l) th_hi = c;
                     }
-                    below = th_hi;  // the (K_l+1)-th score equals the K_l-th
+                    int gt = 0, eq = 0;
+                    uint32_t below = 0;  // largest score word under th_hi: the (K_l+1)-th score if no tie
+                    for (int t = s0; t < s1; ++t) {
+                        const uint32_t h = static_cast<uint32_t>(keys[t] >> 32);
+                        gt += h > th_hi;
+                        eq += h == th_hi;
+                        if (h < th_hi) below = max(below, h);
+                    }
+                    gt = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, gt));
+                    eq = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, eq));
+                    below = __reduce_max_sync(0xFFFFFFFFu, below);
+                    const int need = k_l - gt;  // kept among the keys whose score word is th_hi
+                    th_lo = 0;
+                    if (eq > need) {
+                        // equal scores at the cut: the `need` largest index words (lower nodes)
+                        for (int bit = 31; bit >= 0; --bit) {
+                            const uint32_t c = th_lo | (1u << bit);
+                            int cnt = 0;
+                            for (int t = s0; t < s1; ++t) {
+                                const uint64_t key = keys[t];
+                                cnt += static_cast<uint32_t>(key >> 32) == th_hi && static_cast<uint32_t>(key) >= c;
+                            }
+                            if (static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, cnt)) >= need) th_lo = c;
+                        }
+                        below = th_hi;  // the (K_l+1)-th score equals the K_l-th
+                    }
+                    if (lane == 0) {
+                        const float a = order_bits_inv(th_hi);
+                        const float c = order_bits_inv(below);
+                        const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
+                        s_margin = fminf(s_margin, rel);
+                    }
                 }
-                if (tid == 0) {
-                    const float a = order_bits_inv(th_hi);
-                    const float c = order_bits_inv(below);
-                    const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
-                    s_margin = fminf(s_margin, rel);
-                }
-            }
-            const uint64_t th = (static_cast<uint64_t>(th_hi) << 32) | th_lo;
-            // stable compaction of the kept candidates
-            int mine = 0;
-            for (int t = s0; t < s1; ++t) mine += keys[t] >= th;
-            int incl = mine;
+                const uint64_t th = (static_cast<uint64_t>(th_hi) << 32) | th_lo;
+                // stable compaction of the kept candidates
+                int mine = 0;
+                for (int t = s0; t < s1; ++t) mine += keys[t] >= th;
+                int incl = mine;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += y;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                int pos = incl - mine;
+                for (int t = s0; t < s1; ++t)
+                    if (keys[t] >= th) kept[pos++] = cand[t];
+                if (lane == 31) s_scan[0] = incl;  // how many are kept
             }
-            if (lane == 31) s_scan[warp] = incl;
-            __syncthreads();
-            int pos = incl - mine;
-            for (int w = 0; w < warp; ++w) pos += s_scan[w];
-            const int nkeep = s_scan[0] + s_scan[1] + s_scan[2] + s_scan[3];
-            for (int t = s0; t < s1; ++t)
-                if (keys[t] >= th) kept[pos++] = cand[t];
-            __syncthreads();  // kept[] complete; s_nvalid and s_scan read by every thread
+            __syncthreads();  // kept[] complete; s_nvalid read by every thread
+            const int nkeep = s_scan[0];
             if (l > 0) {
                 // the next candidates: children of the kept parents, parents ascending
                 const int64_t last_below = last / p.width[l - 1];
