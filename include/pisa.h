@@ -209,7 +209,9 @@ PISA_API pisa_status pisa_backward_workspace_size(const pisa_shape *shape, size_
  *   Q, K, V, O : bf16 as in pisa_sparse_attention (O its output), device.
  *   lse        : fp32 [batch, heads_q, seq_q], the forward's LSE, device.
  *   dO         : bf16, same layout as O, device.
- *   idx        : the selection the forward used (same rules on invalid entries).
+ *   idx        : the selection the forward used. Entries < 0, >= n0, or > i when causal are
+ *                skipped (not recorded: the forward call that produced or checked idx records
+ *                them).
  *   dQ, dK, dV : bf16 outputs, the layouts of Q, K, V, device. Every element is written (keys
  *                no query uses get 0).
  *   ws         : >= pisa_backward_workspace_size bytes, 16-byte aligned, device.
