@@ -136,3 +136,42 @@ def test_attention_pair_count_by_brute_force():
                     if j >= 0:
                         brute += sum(1 for key in range(j * 64, j * 64 + 64) if key <= q)
     assert pisa.attention_pairs(idx, s) == brute
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("name", ["tiny", "causal32k", "gqa128k"])
+def test_backward_workspace_layout(name):
+    """Status word, Delta per query row, list offsets per key block, list entries, and the
+    per-range counts of the parallel list fill (32 ranges of query blocks)."""
+    s = shape_of(name)
+    n0, nqb, g = s.n_blocks, s.n_qblocks, s.heads_q // s.heads_kv
+    rsize = -(-nqb // 32)
+    nranges = -(-nqb // rsize)
+    o = 256
+    o = _align256(o + s.batch * s.heads_q * s.seq_q * 4)
+    o = _align256(o + s.batch * s.heads_kv * (n0 + 1) * 4)
+    o = _align256(o + s.batch * s.heads_kv * nqb * s.topk * g * 4)
+    o = _align256(o + s.batch * s.heads_kv * nranges * n0 * 4)
+    assert pisa.backward_workspace_size(s) == o
+
+
+def test_backward_argument_checks():
+    s = shape_of("tiny")
+    c = s.c()
+    f = pisa._lib
+    need = pisa.backward_workspace_size(s)
+    args = [FAKE] * 10
+    assert f.pisa_sparse_attention_backward(ctypes.byref(c), *args, FAKE, need - 1, None) == pisa.ERR_WORKSPACE
+    for k in range(10):
+        bad = list(args)
+        bad[k] = None
+        assert f.pisa_sparse_attention_backward(ctypes.byref(c), *bad, FAKE, need, None) == pisa.ERR_INVALID_ARG
+        bad[k] = MISALIGNED
+        assert f.pisa_sparse_attention_backward(ctypes.byref(c), *bad, FAKE, need, None) == pisa.ERR_INVALID_ARG
+    assert f.pisa_sparse_attention_backward(ctypes.byref(c), *args, None, need, None) == pisa.ERR_INVALID_ARG
+    dec = shape_of("decode128k").c()
+    n = ctypes.c_size_t()
+    assert f.pisa_backward_workspace_size(ctypes.byref(dec), ctypes.byref(n)) == pisa.ERR_UNSUPPORTED

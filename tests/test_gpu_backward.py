@@ -36,9 +36,11 @@ def _grads(w, cuda_device, per_qhead=False, forced=0):
     o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
     g = torch.Generator(device="cpu").manual_seed(w.seed + 1000)
     do = torch.randn(tuple(q.shape), generator=g).to(torch.bfloat16).to(cuda_device)
-    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx)
+    ws_b = torch.zeros(pisa.backward_workspace_size(shape), dtype=torch.uint8, device=cuda_device)
+    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx, ws=ws_b)
     torch.cuda.synchronize()
     pisa.raise_on_device_error(ws)
+    pisa.raise_on_device_error(ws_b, "backward")  # the backward kernels' status word
     return shape, (q, k, v, o, lse, do, idx), (dq, dk, dv)
 
 

@@ -126,9 +126,11 @@ def test_gqa128k_backward_sampled(cuda_device):
     gen = torch.Generator(device="cpu").manual_seed(w.seed + 1000)
     do_h = torch.randn(tuple(q.shape), generator=gen).to(torch.bfloat16)
     do = do_h.to(cuda_device)
-    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx)
+    ws_b = torch.zeros(pisa.backward_workspace_size(shape), dtype=torch.uint8, device=cuda_device)
+    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx, ws=ws_b)
     torch.cuda.synchronize()
-    pisa.raise_on_device_error(ws, "backward")
+    pisa.raise_on_device_error(ws, "forward")
+    pisa.raise_on_device_error(ws_b, "backward")
     del o, lse, q, k, v
     idx_h = idx.cpu().numpy()
     B, g, blk, nqb = 0, w.group, w.block, shape.n_qblocks
