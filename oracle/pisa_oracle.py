@@ -5,7 +5,7 @@ only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg do. It shares no code with the CUDA library.
 
 What it follows (the pages give no equations, pseudo-code or constants; each
-open point takes the plainest reading, listed as R1..R13 in the design notes):
+open point takes the plainest reading, listed as R1..R18 in the design notes):
 
 * "Attention clairsemee PISA : noyaux Triton sans matrice de scores"
   (irisproject.cloud), sections "Une pyramide de cles plutot qu'un tapis
@@ -24,6 +24,15 @@ open point takes the plainest reading, listed as R1..R13 in the design notes):
 * "Dropping the Anchor ... via Pulsar Attention" (gist.science), section
   "Phase 2 : Encodage de la requete globale": partial attentions over disjoint
   key sets are combined by an online-softmax merge  ->  ``merge_partials``.
+* PISA page, section "La selection top-K guidee par la pyramide" (top-K variants
+  may be tuned per domain) and the Pulsar page's fixed attention-sink prefix:
+  blocks that are always kept (sink, local)  ->  ``forced_set`` and the
+  ``forced`` argument of ``select_blocks``.
+* PISA page, section "Ce que cela change pour vous" (memory stays flat as the
+  context grows): a pyramid over a KV cache with spare capacity, every node the
+  mean of the keys it covers among the valid rows  ->  ``build_pyramid_capacity``.
+* same section (the sparse kernels also serve training): gradients of the
+  attention step through a fixed selection  ->  ``attend_backward``, ``backward``.
 
 Parity pins (tests/test_oracle_pins.py) tie every function here to a closed
 form, a brute-force computation or an invariant; none is "parity unpinned".
