@@ -28,11 +28,14 @@ open point takes the plainest reading, listed as R1..R18 in the design notes):
   may be tuned per domain) and the Pulsar page's fixed attention-sink prefix:
   blocks that are always kept (sink, local)  ->  ``forced_set`` and the
   ``forced`` argument of ``select_blocks``.
-* PISA page, section "Ce que cela change pour vous" (memory stays flat as the
-  context grows): a pyramid over a KV cache with spare capacity, every node the
-  mean of the keys it covers among the valid rows  ->  ``build_pyramid_capacity``.
-* same section (the sparse kernels also serve training): gradients of the
-  attention step through a fixed selection  ->  ``attend_backward``, ``backward``.
+* PISA page, section "Des noyaux Triton qui ne materialisent rien" (the memory
+  footprint stays stable as the context grows): a pyramid over a KV cache with
+  spare capacity, every node the mean of the keys it covers among the valid
+  rows  ->  ``build_pyramid_capacity``.
+* PISA page, section "Ce que cela change pour vous" (for those who train as well
+  as deploy models) and the key points' "training as well as inference":
+  gradients of the attention step through a fixed selection  ->
+  ``attend_backward``, ``backward``.
 
 Parity pins (tests/test_oracle_pins.py) tie every function here to a closed
 form, a brute-force computation or an invariant; none is "parity unpinned".
