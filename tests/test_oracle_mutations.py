@@ -122,6 +122,37 @@ def _backward_dk_unscaled(q_rows, q_pos, k_plane, v_plane, blocks, block, causal
     return dq, dk / scale, dv
 
 
+def _backward_with_slip(slip):
+    """The oracle's backward restated with one planted slip."""
+    def bad(q_rows, q_pos, k_plane, v_plane, blocks, block, causal, scale, d_out):
+        if slip == "no_mask":
+            return _orig_attend_backward(q_rows, q_pos, k_plane, v_plane, blocks, block, False, scale, d_out)
+        dq = np.zeros(q_rows.shape)
+        dk = np.zeros(k_plane.shape)
+        dv = np.zeros(v_plane.shape)
+        if len(blocks) == 0:
+            return dq, dk, dv
+        key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
+        q = q_rows.astype(np.float64)
+        kx = k_plane[key_pos].astype(np.float64)
+        vx = v_plane[key_pos].astype(np.float64)
+        do = d_out.astype(np.float64)
+        s = scale * (q @ kx.T)
+        if causal:
+            s = np.where(key_pos[None, :] > q_pos[:, None], -np.inf, s)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ vx
+        dp = do @ vx.T
+        ds = p * (dp - (do * o).sum(axis=1, keepdims=True))
+        dvx = (ds if slip == "dv_from_ds" else p).T @ do
+        dq = scale * (ds @ (vx if slip == "dq_from_v" else kx))
+        np.add.at(dk, key_pos, scale * (ds.T @ q))
+        np.add.at(dv, key_pos, dvx)
+        return dq, dk, dv
+    return bad
+
+
 def _one_level_too_many(n0, factor):
     sizes = [n0]
     while sizes[-1] >= factor:
@@ -148,6 +179,9 @@ MUTATIONS = {
     "capacity pyramid averages the spare rows": ("build_pyramid_capacity", _capacity_counts_spare_blocks),
     "backward drops the row term of dS": ("attend_backward", _backward_no_delta),
     "backward leaves the scale out of dK": ("attend_backward", _backward_dk_unscaled),
+    "backward ignores the causal mask": ("attend_backward", _backward_with_slip("no_mask")),
+    "backward forms dV from dS instead of P": ("attend_backward", _backward_with_slip("dv_from_ds")),
+    "backward multiplies dS by V for dQ": ("attend_backward", _backward_with_slip("dq_from_v")),
 }
 
 
@@ -162,3 +196,12 @@ def test_planted_mistake_is_caught(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin_name)
     assert failed, f"no pin caught: {name}"
+
+
+def test_restated_backward_without_a_slip_passes(monkeypatch):
+    """Control for the backward slips above: the same restatement with no slip passes every pin,
+    so what those mutations trip is the slip, not the restatement."""
+    monkeypatch.setattr(po, "attend_backward", _backward_with_slip("none"))
+    for pin_name, pin in pins.ALL_PINS.items():
+        if pin_name.startswith("backward"):
+            pin(po)
