@@ -175,3 +175,35 @@ def test_backward_argument_checks():
     dec = shape_of("decode128k").c()
     n = ctypes.c_size_t()
     assert f.pisa_backward_workspace_size(ctypes.byref(dec), ctypes.byref(n)) == pisa.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bad", [
+    dict(forced_blocks=4),                                    # unknown variant bit
+    dict(seq_q=1, kv_capacity=4096 - 64),                     # capacity below seq_kv
+    dict(seq_q=1, kv_capacity=8192 + 32),                     # capacity not a multiple of the block
+    dict(kv_capacity=8192),                                   # spare capacity is a decode feature
+])
+def test_selection_variant_and_capacity_checks(bad):
+    s = shape_of("tiny", **bad)
+    n = ctypes.c_size_t()
+    assert pisa._lib.pisa_workspace_size(ctypes.byref(s.c()), ctypes.byref(n)) == pisa.ERR_INVALID_ARG
+
+
+def test_capacity_sets_the_pyramid_layout():
+    s = shape_of("tiny", seq_q=1, kv_capacity=4 * 4096)
+    sizes, offs = pisa.level_layout(s)
+    assert sizes == oracle.level_sizes(4 * 4096 // s.block, s.factor)
+    assert pisa.pyramid_size(s) == s.batch * s.heads_kv * sum(sizes) * s.head_dim * 4
+    for forced in (1, 2, 3):
+        assert pisa.workspace_size(shape_of("tiny", forced_blocks=forced)) > 0
+
+
+def test_append_pyramid_argument_checks():
+    s = shape_of("tiny", seq_q=1, kv_capacity=2 * 4096).c()
+    f = pisa._lib
+    assert f.pisa_append_pyramid(ctypes.byref(s), None, FAKE, 0, None) == pisa.ERR_INVALID_ARG
+    assert f.pisa_append_pyramid(ctypes.byref(s), FAKE, None, 0, None) == pisa.ERR_INVALID_ARG
+    assert f.pisa_append_pyramid(ctypes.byref(s), MISALIGNED, FAKE, 0, None) == pisa.ERR_INVALID_ARG
+    assert f.pisa_append_pyramid(ctypes.byref(s), FAKE, MISALIGNED, 0, None) == pisa.ERR_INVALID_ARG
+    for old in (-64, 4096 + 64, 32):  # negative, past seq_kv, not a whole block
+        assert f.pisa_append_pyramid(ctypes.byref(s), FAKE, FAKE, old, None) == pisa.ERR_INVALID_ARG
