@@ -42,6 +42,7 @@ form, a brute-force computation or an invariant; none is "parity unpinned".
 """
 from __future__ import annotations
 
+import itertools
 import math
 
 import numpy as np
@@ -239,6 +240,99 @@ def select_blocks(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk:
     return {"idx": sorted(kept + forced), "margin": margin, "n_scored": n_scored}
 
 
+def _near(a: float, b: float, rel_tol: float) -> bool:
+    """Two scores within the near-tie tolerance of each other (R10's relative measure)."""
+    return abs(a - b) <= rel_tol * max(abs(a), abs(b), 1e-30)
+
+
+def selection_is_admissible(qbar: np.ndarray, levels: list[np.ndarray], factor: int, topk: int, last: int,
+                            row, budgets: list[int] | None = None, forced: list[int] | None = None,
+                            rel_tol: float = NEAR_TIE_REL, max_branches: int = 4096) -> tuple[bool, str]:
+    """Whether a selection row computed elsewhere is one the descent of ``select_blocks`` can reach
+    when every near-tie at a pruning level may be resolved either way (R10).
+
+    ``row`` lists kept level-0 blocks in ascending order, then -1 padding (R12). It must be well
+    formed: no entry after the padding, strictly ascending (so distinct), every block eligible
+    (0 <= j <= last) and every forced block present (R16). Then the descent is replayed with this
+    oracle's fp32 scores: at a pruning level whose K_l-th and (K_l+1)-th scores are within
+    ``rel_tol`` of each other (a near-tie), the candidates whose scores lie within ``rel_tol`` of
+    either form a band, those above the band are kept, those below it dropped, and any choice of
+    band members that fills the budget is one branch; a level without a near-tie keeps its top
+    K_l. With ``rel_tol = 0`` the branches are exactly the ways of breaking equal scores. The row is
+    admissible if some branch ends with exactly its blocks. Branches are pruned by the row itself:
+    every ancestor j // f^l of a row block must be kept at level l. With no near-tie at any level
+    there is one branch, so the row is admissible exactly when it equals ``select_blocks``'s.
+    Returns (admissible, reason when not).
+    """
+    n_levels = len(levels)
+    n0 = levels[0].shape[0]
+    if budgets is None:
+        budgets = [topk] * n_levels
+    forced = [] if forced is None else list(forced)
+    row = [int(x) for x in row]
+    n_valid = next((t for t, x in enumerate(row) if x < 0), len(row))
+    valid = row[:n_valid]
+    if any(x >= 0 for x in row[n_valid:]):
+        return False, "a block after the -1 padding"
+    if any(valid[t] >= valid[t + 1] for t in range(len(valid) - 1)):
+        return False, "blocks not strictly ascending (unsorted or repeated)"
+    if any(j > last or j >= n0 for j in valid):
+        return False, "a block that is not eligible"
+    if any(f not in valid for f in forced):
+        return False, "a forced block is missing"
+    target = set(valid) - set(forced)
+    top = n_levels - 1
+    start = [c for c in range(levels[top].shape[0]) if node_span(n0, factor, top, c)[0] <= last]
+    stack = [(top, start)]
+    explored = 0
+    while stack:
+        l, cands = stack.pop()
+        explored += 1
+        if explored > max_branches:
+            return False, "more near-tie branches than the search allows"
+        if l == 0 and forced:
+            cands = [c for c in cands if c not in forced]
+        need = {j // factor ** l for j in target}
+        if not need <= set(cands):
+            continue
+        k_l = budgets[l] - (len(forced) if l == 0 else 0)
+        if k_l <= 0:
+            options = [[]]
+        elif len(cands) <= k_l:
+            options = [list(cands)]
+        else:
+            sc = {c: float(score(qbar, node_value(levels, factor, l, c, last))) for c in cands}
+            order = sorted(cands, key=lambda c: rank_key(sc[c], c))
+            s_k, s_k1 = sc[order[k_l - 1]], sc[order[k_l]]
+            band = []
+            if _near(s_k, s_k1, rel_tol):
+                band = [c for c in order if _near(sc[c], s_k, rel_tol) or _near(sc[c], s_k1, rel_tol)]
+            sure = [c for c in order[:k_l] if c not in band]
+            free = k_l - len(sure)
+            if not (need - set(band)) <= set(sure):
+                continue
+            must = [c for c in band if c in need]
+            rest = [c for c in band if c not in need]
+            if len(must) > free:
+                continue
+            if l == 0:
+                options = [sure + must] if len(must) == free else []
+            else:
+                if math.comb(len(rest), free - len(must)) > max_branches:
+                    return False, "more near-tie branches than the search allows"
+                options = [sure + must + list(extra) for extra in itertools.combinations(rest, free - len(must))]
+        for kept in options:
+            if l == 0:
+                if set(kept) == target:
+                    return True, ""
+                continue
+            n_below = levels[l - 1].shape[0]
+            nxt = sorted(ch for c in kept for ch in children(n_below, factor, c)
+                         if node_span(n0, factor, l - 1, ch)[0] <= last)
+            stack.append((l - 1, nxt))
+    return False, "no resolution of the near-ties at the pruning levels gives this row"
+
+
 # ----------------------------------------------------------------------------- attention
 
 def attend(q_rows: np.ndarray, q_pos: np.ndarray, k_plane: np.ndarray, v_plane: np.ndarray,
@@ -415,10 +509,12 @@ def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int, factor: int
     idx = np.full((B, hsel, nqb, topk), -1, dtype=np.int32)
     margin = np.full((B, hsel, nqb), np.inf, dtype=np.float64)
     n_scored = np.zeros((B, hsel, nqb), dtype=np.int64)
+    qbars = np.zeros((B, hsel, nqb, D), dtype=F32)
     for b in range(B):
         for hs in range(hsel):
             kvh, heads = selection_heads(Hq, Hkv, per_qhead, hs)
             qbar = query_summary(Q[b, heads], 1 if decode else block)
+            qbars[b, hs] = qbar
             for i in range(nqb):
                 last = n0 - 1 if (decode or not causal) else i
                 fset = forced_set(forced, n0 - 1 if decode else i, topk)
@@ -441,4 +537,5 @@ def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int, factor: int
                                causal and not decode, sc)
                 O[b, h, rows] = o
                 lse[b, h, rows] = ls
-    return {"O": O, "lse": lse, "idx": idx, "margin": margin, "n_scored": n_scored, "pyramid": pyr}
+    return {"O": O, "lse": lse, "idx": idx, "margin": margin, "n_scored": n_scored, "pyramid": pyr,
+            "qbar": qbars}

@@ -3,7 +3,9 @@ references on the host, and the acceptance checks.
 
 Acceptance (bf16 inputs, fp32 accumulation):
   * selected indices bit-exact, except query blocks whose oracle margin at a
-    pruning level is below 1e-3 (near-ties), which are counted;
+    pruning level is below 1e-3 (near-ties), which are counted; a row that
+    differs must still be well formed and reachable by the descent with its
+    near-ties resolved the other way (``check_selection``);
   * O within max-abs 2e-2 and mean-abs 2e-3 of the oracle run on the GPU's own
     indices; LSE within 1e-3;
   * pyramid within 1e-5 absolute + 1e-5 relative.
@@ -25,11 +27,36 @@ def host_f32(t):
     return t.float().cpu().numpy()
 
 
-def selection_report(gpu_idx, ref_idx, ref_margin):
-    """(mismatching rows that are not near-ties, near-tie rows) over rows given as arrays [..., K]."""
-    same = np.all(gpu_idx == ref_idx, axis=-1)
-    near = np.asarray(ref_margin) < NEAR_TIE
-    return int(np.sum(~same & ~near)), int(np.sum(near))
+def check_selection(gpu_idx, ref, w, *, per_qhead=False, budgets=None, forced=0, topk=None, kv_len=None,
+                    what=""):
+    """Selection rows from the GPU against the oracle's `ref` (``oracle.forward`` on the same inputs).
+
+    A row equal to the oracle's passes. A row that differs must be one the oracle's descent can
+    reach when near-ties (R10) are resolved the other way: ``oracle.selection_is_admissible``
+    checks that it is well formed (min(K, eligible) distinct ascending eligible blocks, then -1,
+    forced blocks present) and replays the descent with every near-tie band open. Any other
+    difference fails the test. Returns (near-tie rows, rows that differ) and prints both.
+    """
+    import oracle
+    topk = w.topk if topk is None else topk
+    g = w.heads_q // w.heads_kv
+    n0 = (w.seq_kv if kv_len is None else kv_len) // w.block
+    gpu_idx = np.asarray(gpu_idx)
+    same = np.all(gpu_idx == ref["idx"], axis=-1)
+    near = np.asarray(ref["margin"]) < NEAR_TIE
+    bad = []
+    for (b, hs, i) in zip(*np.nonzero(~same)):
+        kvh = hs // g if per_qhead else hs
+        last = n0 - 1 if (w.decode or not w.causal) else int(i)
+        fset = oracle.forced_set(forced, n0 - 1 if w.decode else int(i), topk)
+        ok, why = oracle.selection_is_admissible(ref["qbar"][b, hs, i], ref["pyramid"][b][kvh], w.factor, topk,
+                                                 last, gpu_idx[b, hs, i], budgets=budgets, forced=fset)
+        if not ok:
+            bad.append(((int(b), int(hs), int(i)), why, gpu_idx[b, hs, i].tolist(), ref["idx"][b, hs, i].tolist()))
+    n_near, n_diff = int(near.sum()), int((~same).sum())
+    print(f"selection {what or w.name}: {same.size} rows, {n_near} near-ties, {n_diff} differ from the oracle")
+    assert not bad, f"{len(bad)} selection rows not reachable by the descent: {bad[:3]}"
+    return n_near, n_diff
 
 
 def assert_output_close(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
