@@ -67,6 +67,7 @@ _sig = {
     "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pisa_last_launch_count": (ctypes.c_int32, []),
     "pisa_decode_attention_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "pisa_decode_noalloc_check_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -274,6 +275,14 @@ def decode_attention_noalloc(shape: Shape, Q, K, V, idx, O=None, lse=True, strea
     _check(_lib.pisa_decode_attention_noalloc(ctypes.byref(shape.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                               _ptr(O), _ptr(L), _stream(stream)), "pisa_decode_attention_noalloc")
     return O, L
+
+
+def decode_noalloc_check_status(stream=None) -> tuple[int, int]:
+    """Synchronises the stream; returns (status, detail) that the last decode_attention_noalloc
+    call's kernels recorded in the library's built-in array, and clears them."""
+    detail = ctypes.c_uint32()
+    st = _lib.pisa_decode_noalloc_check_status(ctypes.byref(detail), _stream(stream))
+    return int(st), int(detail.value)
 
 
 def backward_workspace_size(shape: Shape) -> int:

@@ -9,14 +9,19 @@
 // Every GPU that loads the library holds that array until the process exits.
 //
 // Host code cannot pass the array's name to a kernel (on the host it only
-// stands in for the symbol), so the first call on each device looks up its
-// device address with cudaGetSymbolAddress, with that device current, and
-// keeps it. Every call on a device shares the one array: two calls whose
-// kernels overlap on the GPU (different streams, no ordering between them)
-// race on it.
+// stands in for the symbol), so every call looks up its device address with
+// cudaGetSymbolAddress, with the calling device current. The lookup allocates
+// nothing; doing it per call (rather than caching the address) keeps it right
+// after the device's context is torn down and created again. The first call on
+// a device may load the library's device code there, so it should come before
+// any stream capture. Every call on a
+// device shares the one array: two calls whose kernels overlap on the GPU
+// (different streams, no ordering between them) race on it.
+//
+// Each call clears the array's status word before its kernels run; the
+// kernels record an out-of-range block index or a pipeline wait that ran out
+// of time there, and pisa_decode_noalloc_check_status reads and clears it.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "pisa.h"
 #include "pisa_internal.h"
@@ -24,28 +29,12 @@
 namespace pisa {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
-constexpr int kNoAllocMaxDevices = 256;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_addr[kNoAllocMaxDevices];
-
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array on the current device.
 static cudaError_t noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
-    return cudaSuccess;
+    return cudaGetSymbolAddress(out, g_noalloc_scratch);
 }
 
 }  // namespace pisa
@@ -70,7 +59,8 @@ extern "C" pisa_status pisa_decode_attention_noalloc(const pisa_shape* shape, co
     void* scratch = nullptr;
     if (noalloc_scratch(&scratch) != cudaSuccess) return PISA_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // the status word keeps the previous call's contents: it must start at zero
+    // the array keeps the previous call's contents: the status word must start at zero (the
+    // partials need no clearing: every split writes its partial before the merge reads it)
     if (cudaMemsetAsync(scratch, 0, kStatusBytes, st) != cudaSuccess) return PISA_ERR_CUDA;
 
     DecodeParams d{};
@@ -98,4 +88,19 @@ extern "C" pisa_status pisa_decode_attention_noalloc(const pisa_shape* shape, co
     d.scale_log2 = pl.scale * 1.4426950408889634f;
     int32_t launches = 0;
     return launch_attn_decode(pl, d, st, &launches) ? PISA_OK : PISA_ERR_CUDA;
+}
+
+extern "C" pisa_status pisa_decode_noalloc_check_status(uint32_t* detail, pisa_stream_t stream) {
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return PISA_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t host[2] = {0, 0};
+    if (cudaMemcpyAsync(host, scratch, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess) return PISA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+    if (host[0] != 0) {
+        if (cudaMemsetAsync(scratch, 0, sizeof(host), st) != cudaSuccess) return PISA_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+    }
+    if (detail) *detail = host[1];
+    return static_cast<pisa_status>(host[0]);
 }

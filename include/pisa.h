@@ -240,20 +240,34 @@ PISA_API pisa_status pisa_forward(const pisa_shape *shape, const void *Q, const 
  * a caller workspace. The caller still passes Q, K, V, idx, O and lse (lse may
  * be NULL), laid out as for pisa_sparse_attention.
  *   - Every GPU that loads the library holds the 8 MiB array until exit.
- *   - The first call on a device looks up the array's device address with that
- *     device current and keeps it; make that first call before any stream
- *     capture.
- *   - Shapes whose partials need more than the array holds (batch x Hsel x
- *     ceil(topk/4) x g x (head_dim+2) x 4 bytes, plus 256) return
- *     PISA_ERR_WORKSPACE; non-decode shapes return PISA_ERR_INVALID_ARG.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *     which allocates nothing) with the calling device current. The first
+ *     call on a device may load the library's device code there: make it
+ *     before any stream capture.
+ *   - Size limit: with rows = batch * Hsel (Hsel = heads_kv, or heads_q with
+ *     select_per_qhead), gsel = heads_q / heads_kv (1 with select_per_qhead),
+ *     per_split = clamp(ceil(topk / ceil(592 / rows)), 2, 16) and
+ *     splits = ceil(topk / per_split), the call needs
+ *     256 + rows * splits * gsel * (head_dim + 2) * 4 bytes <= 8 MiB; a larger
+ *     shape returns PISA_ERR_WORKSPACE. (64 sequences, 8 KV heads, 32 query
+ *     heads, head_dim 128, topk 64: 4 splits, 4.26 MB.) Non-decode shapes
+ *     return PISA_ERR_INVALID_ARG.
  *   - Calls share the array: calls whose kernels overlap on the GPU race on it.
- *     The status word is cleared at the start of each call; errors the kernels
- *     record there are not reported, and pisa_last_launch_count does not count
- *     this call.
+ *     Each call clears the status word when it starts; errors its kernels
+ *     record there (an idx entry outside [0, n0), a pipeline wait that ran out
+ *     of time) are read by pisa_decode_noalloc_check_status.
+ *     pisa_last_launch_count does not count this call.
  *   - No cudaMalloc, cudaFree or allocating library routine is called. */
 PISA_API pisa_status pisa_decode_attention_noalloc(const pisa_shape *shape, const void *Q, const void *K,
                                                    const void *V, const int32_t *idx, void *O, float *lse,
                                                    pisa_stream_t stream);
+
+/* Companion of pisa_decode_attention_noalloc (no counterpart in the paper either):
+ * synchronises `stream`, returns the device-side error the most recent
+ * pisa_decode_attention_noalloc call on the current device recorded in the
+ * library's array (PISA_OK if none) and clears it. `detail`, if not NULL,
+ * receives the code locating the error. Allocates nothing. */
+PISA_API pisa_status pisa_decode_noalloc_check_status(uint32_t *detail, pisa_stream_t stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace status word since the last call (PISA_OK if none) and clears it.
