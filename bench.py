@@ -59,16 +59,17 @@ ATTN_SOURCES = ("block_sparse_long_pisa_b200/csrc/attn_prefill.cu", "block_spars
 
 
 def profiled_traffic(kernel_file: str, sources) -> float | None:
-    """dram bytes per launch recorded by an ncu capture summary (profiles/<file>), or None when
-    absent or when the kernel sources have changed since the capture (sha256 prefix recorded there)."""
+    """dram bytes per full-size launch recorded from an ncu capture (profiles/<file>, JSON), or None
+    when absent or when the kernel sources have changed since the capture (sha256 prefix recorded
+    there)."""
     p = os.path.join(ROOT, "profiles", kernel_file)
     if not os.path.exists(p):
         return None
-    sha = kernel_source_hash(sources)
-    fields = dict(line.split(":", 1) for line in open(p) if ":" in line and not line.startswith((" ", "|", "#")))
-    if fields.get("source_sha256_16", "").strip() != sha:
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("source_sha256_16") != kernel_source_hash(sources):
         return None
-    v = fields.get("dram_bytes_per_launch_full_size")
+    v = rec.get("dram_bytes_per_launch_full_size")
     return float(v) if v is not None else None
 
 
@@ -180,10 +181,11 @@ def oracle_sample(w, budget_s: float = 15.0) -> dict:
     nqb = w.seq_q // w.block
     rng = np.random.Generator(np.random.PCG64(0))
     order = [nqb - 1] + [int(x) for x in rng.permutation(nqb - 1)]
-    sel = {}
+    sel, margin = {}, {}
     t0 = time.perf_counter()
     for i in order:
-        sel[i] = oracle.select_blocks(qbar[i], levels, w.factor, w.topk, i if w.causal else nqb - 1)["idx"]
+        r = oracle.select_blocks(qbar[i], levels, w.factor, w.topk, i if w.causal else nqb - 1)
+        sel[i], margin[i] = r["idx"], r["margin"]
         if time.perf_counter() - t0 > budget_s / 3:
             break
     t_sel = (time.perf_counter() - t0) / len(sel)
@@ -210,7 +212,42 @@ def oracle_sample(w, budget_s: float = 15.0) -> dict:
                        f"query blocks ({t_sel * 1e3:.1f} ms each), attention of {n_att} of them x {w.group} heads "
                        f"({t_att * 1e3:.1f} ms each); extrapolated to {units} KV heads x {nqb} query blocks"),
             "seconds": round(t_pool + t_sel * len(sel) + t_att * n_att, 1),
-            "estimated_full_seconds": round(total, 1)}
+            "estimated_full_seconds": round(total, 1),
+            "_sample": {"levels": levels, "qbar": qbar, "sel": sel, "margin": margin}}
+
+
+def check_sampled_selection(w, sample: dict, gpu_rows) -> dict:
+    """The oracle rows the CPU-baseline sample computed (KV head 0 of batch 0) against the GPU's
+    rows for the same query blocks: near-ties (oracle margin below 1e-3), rows that differ, and
+    whether each differing row is one the descent reaches with its near-ties resolved the other
+    way (checked by the oracle, outside every timed region)."""
+    import oracle
+    nqb = w.seq_q // w.block
+    near = differ = admissible = 0
+    for i, want in sample["sel"].items():
+        near += sample["margin"][i] < oracle.NEAR_TIE_REL
+        row = [int(x) for x in gpu_rows[i]]
+        if row == list(want) + [-1] * (w.topk - len(want)):
+            continue
+        differ += 1
+        ok, _ = oracle.selection_is_admissible(sample["qbar"][i], sample["levels"], w.factor, w.topk,
+                                               i if w.causal else nqb - 1, row)
+        admissible += ok
+    return {"rows": len(sample["sel"]), "near_ties": int(near), "differ": differ, "differ_admissible": admissible,
+            "sample": "the CPU baseline's descents (KV head 0, random query blocks) vs the GPU's rows"}
+
+
+def needle_recall(w, idx_h) -> dict | None:
+    """Planted needle blocks (16 per KV head) found in their target query block's selection."""
+    if w.keys != "needle":
+        return None
+    found = planted = 0
+    for b in range(w.batch):
+        for kvh in range(w.heads_kv):
+            for (i, j) in workloads.needles(w, b, kvh):
+                planted += 1
+                found += int(j in idx_h[b, kvh, i])
+    return {"planted": planted, "selected": found, "recall": found / planted}
 
 
 def run_reference(args, world, rank):
@@ -223,6 +260,8 @@ def run_reference(args, world, rank):
     t0 = time.perf_counter()
     vals = [oracle_sample(w, budget_s=4.0) for _ in range(args.steps)]
     wall = time.perf_counter() - t0
+    for x in vals:
+        x.pop("_sample")
     v = statistics.median([x["value"] for x in vals])
     base = dict(vals[-1])
     base["value"] = v
@@ -344,12 +383,19 @@ def run_gpu(args, world, rank, local):
                "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": e2e_ms,
                "path": "Session.forward: pinned host Q/K/V -> device, pisa_forward, O -> pinned host"}
 
+    # near-ties over every row from the library's own margins (outside the timed region)
+    _, marg = pisa.select_blocks(shape, q, pyr, ws, margin=True)
+    near_gpu = int((marg < 1e-3).sum().item())
+    pisa.raise_on_device_error(ws, "margins")
     if rank != 0:
         return
     cpu = (oracle_sample(bench_workload(args))
            if world == 1 and not args.no_cpu_baseline and not args.per_qhead else None)
+    near_ties = {"rows": int(marg.numel()), "gpu_margin_below_1e-3": near_gpu}
+    if cpu is not None:
+        near_ties["oracle_sample"] = check_sampled_selection(w, cpu.pop("_sample"), idx_h[0, 0])
     # the recorded ncu traffic belongs to the group-shared launch (two 128-row tiles per CTA)
-    traffic = None if args.per_qhead else profiled_traffic("attn_prefill_gqa128k.md", ATTN_SOURCES)
+    traffic = None if args.per_qhead else profiled_traffic("attn_prefill_gqa128k.json", ATTN_SOURCES)
     config = config_dict(w, world)
     if args.per_qhead:
         config["workload"] += ", per-query-head selection"
@@ -372,6 +418,7 @@ def run_gpu(args, world, rank, local):
                      "peak_source": f"{how} bf16 dense (burst)", "traffic": traffic,
                      "flops_per_launch": attn_flops},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clocks,
+        "near_ties": near_ties, "needle_recall": None if args.per_qhead else needle_recall(w, idx_h),
     }
     print(json.dumps(line), flush=True)
 

@@ -23,3 +23,33 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
+
+
+def test_bench_selection_report_helpers():
+    """The bench's selection report: the CPU baseline's sampled descents compared with given rows
+    (equal rows pass, a doctored row is counted as differing and not admissible), and the needle
+    recall count."""
+    import numpy as np
+    import bench
+    import workloads
+    w = workloads.Workload("bench-needle", 1, 8, 2, 256 * 64, 256 * 64, 64, 64, 4, 16, 1, "needle", 18)
+    cpu = bench.oracle_sample(w, budget_s=1.0)
+    sample = cpu.pop("_sample")
+    nqb = w.seq_q // w.block
+    rows = np.full((nqb, w.topk), -1, dtype=np.int32)
+    for i, sel in sample["sel"].items():
+        rows[i, :len(sel)] = sel
+    rep = bench.check_sampled_selection(w, sample, rows)
+    assert rep["rows"] == len(sample["sel"]) and rep["differ"] == 0
+    i = max(sample["sel"], key=lambda t: len(sample["sel"][t]))
+    assert len(sample["sel"][i]) == w.topk
+    rows[i, 0] = rows[i, 1]            # a repeated block
+    rep = bench.check_sampled_selection(w, sample, rows)
+    assert rep["differ"] == 1 and rep["differ_admissible"] == 0
+    idx = np.full((1, w.heads_kv, nqb, w.topk), -1, dtype=np.int32)
+    for kvh in range(w.heads_kv):
+        for n, (qi, j) in enumerate(workloads.needles(w, 0, kvh)):
+            if n % 2 == 0:
+                idx[0, kvh, qi, 0] = j
+    rec = bench.needle_recall(w, idx)
+    assert rec["planted"] == 16 * w.heads_kv and rec["selected"] == 8 * w.heads_kv
