@@ -68,6 +68,7 @@ _sig = {
     "pisa_last_launch_count": (ctypes.c_int32, []),
     "pisa_decode_attention_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "pisa_decode_noalloc_check_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp]),
+    "pisa_selftest_wait_timeout": (ctypes.c_int, [_vp, ctypes.c_uint32, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -320,6 +321,12 @@ def check_status(ws, stream=None) -> tuple[int, int]:
     return int(st), int(detail.value)
 
 
+def selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:
+    """Enqueues the bounded-wait self-test: a wait that never completes gives up after limit_us
+    and records PISA_ERR_TIMEOUT in the workspace status word (read it with check_status)."""
+    _check(_lib.pisa_selftest_wait_timeout(_ptr(ws), int(limit_us), _stream(stream)), "pisa_selftest_wait_timeout")
+
+
 def raise_on_device_error(ws, where="device", stream=None) -> None:
     st, detail = check_status(ws, stream)
     if st != OK:
@@ -329,37 +336,78 @@ def raise_on_device_error(ws, where="device", stream=None) -> None:
 class Session:
     """Preallocated device buffers for repeated forwards of one shape.
 
-    `forward` accepts host (CPU, ideally pinned) or device tensors. Host inputs
-    are copied to the device on the current stream, the pyramid, selection and
-    attention run in the library, and O is copied back into a host tensor.
+    `forward` accepts host (CPU, ideally pinned) or device tensors. With host
+    inputs the (batch, KV head) planes, which the method treats independently,
+    are split into `units` ranges and pipelined over three streams: the copy
+    of a range's Q, K and V to the device (copy stream), pisa_forward on that
+    range (the caller's current stream) and the copy of its O back to the host
+    (output stream), so that host-device transfers in both directions overlap
+    the computation of other ranges. Each range is one pisa_forward call on a
+    shape with batch = planes in the range, heads_q = g, heads_kv = 1; for
+    prefill its results equal those of one call on the whole shape bit for bit.
     """
 
-    def __init__(self, shape: Shape, device="cuda"):
+    def __init__(self, shape: Shape, device="cuda", units: int = 8):
         torch = _torch()
         self.shape = shape
         self.device = torch.device(device)
         s = shape
         self.ws = new_workspace(shape, self.device)
         self.q = torch.empty((s.batch, s.heads_q, s.seq_q, s.head_dim), dtype=torch.bfloat16, device=self.device)
-        self.k = torch.empty((s.batch, s.heads_kv, s.seq_kv, s.head_dim), dtype=torch.bfloat16, device=self.device)
+        self.k = torch.empty((s.batch, s.heads_kv, s.kv_rows, s.head_dim), dtype=torch.bfloat16, device=self.device)
         self.v = torch.empty_like(self.k)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((s.batch, s.heads_q, s.seq_q), dtype=torch.float32, device=self.device)
+        planes = s.batch * s.heads_kv
+        n = max(1, min(units, planes))
+        bounds = [planes * u // n for u in range(n + 1)]
+        self.ranges = [(a, b) for a, b in zip(bounds, bounds[1:]) if b > a]
+        g = s.heads_q // s.heads_kv
+        self.unit_shapes = {b - a: dataclasses.replace(s, batch=b - a, heads_q=g, heads_kv=1) for a, b in self.ranges}
+        self.unit_ws = new_workspace(max(self.unit_shapes.values(), key=workspace_size), self.device)
+        self.copy_stream = torch.cuda.Stream(self.device)
+        self.out_stream = torch.cuda.Stream(self.device)
+
+    def _planes(self, t, per_plane):
+        """View of a [B, H, ...] tensor as [planes, per_plane, ...] (planes = B * heads_kv)."""
+        return t.view(self.shape.batch * self.shape.heads_kv, per_plane, *t.shape[2:])
 
     def forward(self, Q, K, V, out=None):
-        on_host = not Q.is_cuda
-        if on_host:
-            self.q.copy_(Q, non_blocking=True)
-            self.k.copy_(K, non_blocking=True)
-            self.v.copy_(V, non_blocking=True)
-            Q, K, V = self.q, self.k, self.v
-        O, L, _ = forward(self.shape, Q, K, V, self.ws, O=self.o, lse=self.lse)
-        if on_host:
-            if out is None:
-                out = _torch().empty(tuple(O.shape), dtype=O.dtype, pin_memory=True)
-            out.copy_(O, non_blocking=True)
-            return out
-        return O
+        torch = _torch()
+        if Q.is_cuda:
+            O, _, _ = forward(self.shape, Q, K, V, self.ws, O=self.o, lse=self.lse)
+            return O
+        s = self.shape
+        g = s.heads_q // s.heads_kv
+        if out is None:
+            out = torch.empty(tuple(self.o.shape), dtype=self.o.dtype, pin_memory=True)
+        hq, hk, hv, ho = self._planes(Q, g), self._planes(K, 1), self._planes(V, 1), self._planes(out, g)
+        dq, dk, dv, do = self._planes(self.q, g), self._planes(self.k, 1), self._planes(self.v, 1), self._planes(self.o, g)
+        dl = self.lse.view(s.batch * s.heads_kv, g, s.seq_q)
+        compute = torch.cuda.current_stream(self.device)
+        arrived = []
+        # inputs: every range back to back on the copy stream (after earlier work on these buffers)
+        self.copy_stream.wait_stream(compute)
+        with torch.cuda.stream(self.copy_stream):
+            for a, b in self.ranges:
+                dq[a:b].copy_(hq[a:b], non_blocking=True)
+                dk[a:b].copy_(hk[a:b], non_blocking=True)
+                dv[a:b].copy_(hv[a:b], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.copy_stream)
+                arrived.append(ev)
+        self.out_stream.wait_stream(compute)
+        for (a, b), ev in zip(self.ranges, arrived):
+            compute.wait_event(ev)
+            forward(self.unit_shapes[b - a], dq[a:b], dk[a:b], dv[a:b], self.unit_ws, O=do[a:b], lse=dl[a:b],
+                    stream=compute)
+            done = torch.cuda.Event()
+            done.record(compute)
+            self.out_stream.wait_event(done)
+            with torch.cuda.stream(self.out_stream):
+                ho[a:b].copy_(do[a:b], non_blocking=True)
+        compute.wait_stream(self.out_stream)
+        return out
 
 
 # ----------------------------------------------------------------------------- measurement helpers

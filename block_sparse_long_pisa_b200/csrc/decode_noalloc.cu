@@ -55,6 +55,7 @@ extern "C" pisa_status pisa_decode_attention_noalloc(const pisa_shape* shape, co
     const size_t part_bytes =
         static_cast<size_t>(pl.B) * pl.Hsel * pl.dec_splits * pl.gsel * (pl.D + 2) * sizeof(float);
     if (kStatusBytes + part_bytes > kNoAllocScratchBytes) return PISA_ERR_WORKSPACE;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
 
     void* scratch = nullptr;
     if (noalloc_scratch(&scratch) != cudaSuccess) return PISA_ERR_CUDA;

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "pisa.h"
@@ -98,10 +99,24 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
     p->ws_part = o;
     if (p->decode)
         o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->dec_splits * p->gsel * (p->D + 2) * sizeof(float));
-    p->dense_select = !p->decode && p->nqb >= kDenseSelectMinQBlocks;
+    // dense prefill scoring while its candidate count stays within a few times the sparse
+    // descent's (causal rows see half the nodes on average), in chunks of query blocks whose
+    // score plane fits kSelectPlaneBudget
+    {
+        const int64_t dense = static_cast<int64_t>(p->total_nodes) / (p->causal ? 2 : 1);
+        const int64_t sparse = p->lsize[p->L - 1] + static_cast<int64_t>(p->L - 1) * p->topk * p->f;
+        p->dense_select = !p->decode && p->nqb >= kDenseSelectMinQBlocks &&
+                          dense <= static_cast<int64_t>(kDenseSelectMaxWorkRatio) * sparse;
+    }
     p->ws_scores = o;
-    if (p->dense_select)
-        o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->nqb * p->total_nodes * sizeof(float));
+    if (p->dense_select) {
+        const size_t per128 = size_t(128) * p->B * p->Hsel * p->total_nodes * sizeof(float);
+        const int64_t max_qc = 128 * static_cast<int64_t>(kSelectPlaneBudget / per128 > 0 ? kSelectPlaneBudget / per128 : 1);
+        const int64_t chunks = (p->nqb + max_qc - 1) / max_qc;
+        const int64_t qc = chunks <= 1 ? p->nqb : ((p->nqb + chunks - 1) / chunks + 127) / 128 * 128;
+        p->dense_qc = static_cast<int32_t>(qc);
+        o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->dense_qc * p->total_nodes * sizeof(float));
+    }
     p->ws_total = o;
     return PISA_OK;
 }
@@ -166,8 +181,36 @@ static pisa_status pyramid_range(const Plan& pl, const void* K, float* pyr, int3
     return PISA_OK;
 }
 
+// Whole pyramid: subtrees of S = f^m key blocks (f^m <= max(64, f), m <= L - 1) formed in one
+// launch, the levels above them in a second; a single-level pyramid or a factor above 64 takes
+// the per-level path. Both give the same values bit for bit.
 static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cudaStream_t st) {
-    return pyramid_range(pl, K, pyr, 0, pl.n0_cap, st);
+    if (pl.L < 2 || pl.f > 64) return pyramid_range(pl, K, pyr, 0, pl.n0_cap, st);
+    SubtreeParams p{};
+    p.m = 1;
+    p.S = pl.f;
+    while (p.m + 1 <= pl.L - 1 && static_cast<int64_t>(p.S) * pl.f <= 64) {
+        p.S *= pl.f;
+        ++p.m;
+    }
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.pyr = pyr;
+    p.planes = static_cast<int64_t>(pl.B) * pl.Hkv;
+    p.subtrees = (pl.lsize[0] + p.S - 1) / p.S;
+    if (p.planes * p.subtrees >= (int64_t(1) << 31) || p.planes >= (int64_t(1) << 31))
+        return pyramid_range(pl, K, pyr, 0, pl.n0_cap, st);
+    p.N = pl.N;
+    p.D = pl.D;
+    p.blk = pl.blk;
+    p.factor = pl.f;
+    p.L = pl.L;
+    p.plane_rows = pl.total_nodes;
+    p.n0 = pl.n0;
+    for (int l = 0; l < pl.L; ++l) {
+        p.lsize[l] = pl.lsize[l];
+        p.loff[l] = pl.loff[l];
+    }
+    return launch_pyramid_two_pass(p, st, &g_launches) ? PISA_OK : PISA_ERR_CUDA;
 }
 
 static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cudaStream_t st) {
@@ -222,6 +265,7 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
         w = w > (int64_t(1) << 40) ? w : w * pl.f;
     }
     sp.scores = pl.dense_select ? reinterpret_cast<float*>(ws + pl.ws_scores) : nullptr;
+    sp.qc = pl.dense_qc;
     if (!launch_select(sp, pl.B, st, &g_launches)) return PISA_ERR_CUDA;
     return PISA_OK;
 }
@@ -285,6 +329,11 @@ static pisa_status check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
 
 }  // namespace pisa
 
+bool pisa::injected_launch_failure() {
+    const char* f = getenv("PISA_FAULT");
+    return f != nullptr && strcmp(f, "launch") == 0;
+}
+
 using namespace pisa;
 
 extern "C" {
@@ -328,6 +377,7 @@ pisa_status pisa_build_pyramid(const pisa_shape* shape, const void* K, float* py
     const pisa_status s = make_plan(shape, &pl);
     if (s != PISA_OK) return s;
     if (K == nullptr || pyramid == nullptr || !aligned16(K) || !aligned16(pyramid)) return PISA_ERR_INVALID_ARG;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     return build_pyramid(pl, K, pyramid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -339,6 +389,7 @@ pisa_status pisa_append_pyramid(const pisa_shape* shape, const void* K, float* p
     if (s != PISA_OK) return s;
     if (K == nullptr || pyramid == nullptr || !aligned16(K) || !aligned16(pyramid)) return PISA_ERR_INVALID_ARG;
     if (seq_kv_old < 0 || seq_kv_old > shape->seq_kv || seq_kv_old % pl.blk != 0) return PISA_ERR_INVALID_ARG;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     return pyramid_range(pl, K, pyramid, seq_kv_old / pl.blk, pl.n0, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -399,6 +450,7 @@ pisa_status pisa_sparse_attention_backward(const pisa_shape* shape, const void* 
         if (q == nullptr || !aligned16(q)) return PISA_ERR_INVALID_ARG;
     if (ws == nullptr || !aligned16(ws)) return PISA_ERR_INVALID_ARG;
     if (ws_bytes < w.total) return PISA_ERR_WORKSPACE;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     uint8_t* wb = static_cast<uint8_t*>(ws);
     BwdParams p{};
     p.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -459,6 +511,7 @@ pisa_status pisa_select_blocks(const pisa_shape* shape, const void* Q, const flo
         return PISA_ERR_INVALID_ARG;
     if ((s = check_budget(pl, level_budget)) != PISA_OK) return s;
     if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
@@ -477,6 +530,7 @@ pisa_status pisa_sparse_attention(const pisa_shape* shape, const void* Q, const 
         !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx))
         return PISA_ERR_INVALID_ARG;
     if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     return attention(pl, Q, K, V, idx, O, lse, static_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -490,6 +544,7 @@ pisa_status pisa_forward(const pisa_shape* shape, const void* Q, const void* K, 
         !aligned16(V) || !aligned16(O) || (idx_out != nullptr && !aligned16(idx_out)))
         return PISA_ERR_INVALID_ARG;
     if ((s = check_ws(pl, ws, ws_bytes)) != PISA_OK) return s;
+    if (injected_launch_failure()) return PISA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* pyr = reinterpret_cast<float*>(w + pl.ws_pyramid);

@@ -65,14 +65,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the barrier phase with the given parity has completed. Gives up
-// after kWaitLimitNs, records PISA_ERR_TIMEOUT with `site` and returns false,
-// so that no kernel of this library can spin forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t site) {
+// after `limit_ns` (kWaitLimitNs unless given), records PISA_ERR_TIMEOUT with
+// `site` and returns false, so that no kernel of this library can spin forever.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t site,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             record_error(status, PISA_ERR_TIMEOUT, site);
             return false;
         }

@@ -24,6 +24,14 @@ constexpr int kDecMaxBps = 16;
 // eligible node densely (the tiles are shared by 128 query blocks); fewer
 // query blocks (and decode) score only the descent's candidates.
 constexpr int kDenseSelectMinQBlocks = 16;
+// The dense scoring is used while it scores at most this many times the
+// candidates the sparse descent scores (it is ~5x cheaper per candidate);
+// past that (very long contexts) the sparse descent's O(N log N) work wins.
+constexpr int kDenseSelectMaxWorkRatio = 4;
+// Bytes of score plane one dense-selection pass may hold: the query blocks
+// are scored and descended in chunks whose plane fits this (the 128K GQA
+// prefill fits in one chunk; every chunk costs two more launches).
+constexpr size_t kSelectPlaneBudget = size_t(192) << 20;
 
 // Bytes reserved for the status word at the start of the workspace.
 constexpr size_t kStatusBytes = 256;
@@ -35,7 +43,14 @@ enum : uint32_t {
     kKernAttnDecode = 2,
     kKernSelect = 3,
     kKernAttnBackward = 4,
+    kKernSelftest = 5,
 };
+
+// Fault injection on the host: true when the environment variable PISA_FAULT
+// is "launch". Every enqueuing entry point then returns PISA_ERR_CUDA after
+// its argument checks, as if its first kernel launch had failed, and enqueues
+// nothing (no GPU fault is involved).
+bool injected_launch_failure();
 
 // Derived sizes of one problem (host side).
 struct Plan {
@@ -57,6 +72,7 @@ struct Plan {
     // workspace layout (byte offsets)
     size_t ws_pyramid, ws_qbar, ws_idx, ws_part, ws_scores, ws_total;
     int32_t dense_select;       // prefill selection scores densely (score plane in the workspace)
+    int32_t dense_qc;           // query blocks per dense-selection chunk (a multiple of 128, or nqb)
     size_t pyramid_bytes;
 };
 
@@ -90,6 +106,19 @@ struct LevelParams {
     int64_t width_below;        // level-0 blocks under one node of the level below (f^(l-1))
 };
 
+// Two-launch pyramid build: subtrees of S = factor^m key blocks, then the levels above them.
+struct SubtreeParams {
+    const __nv_bfloat16* K;     // bf16 [planes, N, D]
+    float* pyr;                 // fp32 [planes, plane_rows, D]
+    int64_t planes;             // batch * heads_kv
+    int32_t subtrees;           // ceil(lsize[0] / S) per plane
+    int32_t S, m;               // key blocks per subtree (factor^m) and the levels formed inside it
+    int32_t N, D, blk, factor, L, plane_rows;
+    int32_t n0;                 // level-0 blocks that hold keys (the rest of the capacity is zero)
+    int32_t lsize[PISA_MAX_LEVELS];
+    int32_t loff[PISA_MAX_LEVELS];
+};
+
 struct SelectParams {
     const float* qbar;          // fp32 [B, Hsel, nqb, D]
     const float* pyr;           // fp32 [B, Hkv, total_nodes, D]
@@ -104,7 +133,9 @@ struct SelectParams {
     int32_t loff[PISA_MAX_LEVELS];
     int32_t budget[PISA_MAX_LEVELS];
     int64_t width[PISA_MAX_LEVELS];  // f^l (saturated)
-    float* scores;                   // dense prefill scoring: fp32 [B, Hsel, nqb, total_nodes], or null
+    float* scores;                   // dense prefill scoring: fp32 [B, Hsel, qc, total_nodes], or null
+    int32_t qc;                      // query blocks per dense chunk (plane rows per selection row)
+    int32_t i_lo, nqc;               // the chunk being scored: query blocks [i_lo, i_lo + nqc)
     int32_t tile_off[PISA_MAX_LEVELS + 1];  // score tiles before level l (set by the launcher)
     int32_t tiles_c[PISA_MAX_LEVELS];       // node tiles of level l (set by the launcher)
 };
@@ -159,12 +190,14 @@ struct BwdParams {
 
 bool launch_block_mean(const MeanParams& p, cudaStream_t st);
 bool launch_pyramid_level(const LevelParams& p, cudaStream_t st);
+// Whole pyramid in two launches (adds them to *launches).
+bool launch_pyramid_two_pass(const SubtreeParams& p, cudaStream_t st, int32_t* launches);
 // Launches the selection; adds the kernels it launched to *launches. Prefill
 // with a score plane and candidate sets of at most 1024 runs the dense scoring
 // kernel and the warp descent; otherwise the one-CTA-per-row sparse descent.
 bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
 int dense_select_cap(int cap);
-bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st);
+bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st, int32_t* launches);
 // Prefill attention: builds the tensor maps and picks the kernel variant.
 pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
                                 cudaStream_t st, int32_t* launches);

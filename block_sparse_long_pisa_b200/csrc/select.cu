@@ -293,10 +293,7 @@ bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_
     int cap = 1;
     while (cap < max(p.factor * maxb, p.lsize[p.L - 1])) cap <<= 1;
     if (cap < 4) cap = 4;  // keeps the fp32 query row 16-byte aligned
-    if (p.scores != nullptr && !p.decode && dense_select_cap(cap) > 0) {
-        *launches += 2;
-        return launch_select_dense(p, batch, cap, st);
-    }
+    if (p.scores != nullptr && !p.decode && dense_select_cap(cap) > 0) return launch_select_dense(p, batch, cap, st, launches);
     *launches += 1;
     const size_t smem = static_cast<size_t>(cap) * (sizeof(uint64_t) + 2 * sizeof(int32_t)) +
                         static_cast<size_t>(p.D) * (1 + p.L) * sizeof(float);

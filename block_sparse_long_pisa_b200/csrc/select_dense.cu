@@ -65,9 +65,10 @@ __global__ void __launch_bounds__(kScThreads, 2) score_kernel(const SelectParams
     int tile = blockIdx.x, l = 0;
     while (l + 1 < p.L && tile >= p.tile_off[l + 1]) ++l;
     tile -= p.tile_off[l];
-    const int i0 = (tile / p.tiles_c[l]) * kScTile;
+    const int i_end = p.i_lo + p.nqc;  // this chunk's query blocks: [i_lo, i_end)
+    const int i0 = p.i_lo + (tile / p.tiles_c[l]) * kScTile;
     const int c0 = (tile % p.tiles_c[l]) * kScTile;
-    const int i_hi = min(i0 + kScTile, p.nqb) - 1;
+    const int i_hi = min(i0 + kScTile, i_end) - 1;
     const int64_t last_hi = p.causal ? i_hi : p.n0_valid - 1;
     // the start level and the eligible range only grow with the query block
     if (start_level(p, last_hi) < l || c0 > last_hi / p.width[l]) return;
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kScThreads, 2) score_kernel(const SelectParams
     const int ld_row = tid >> 3, ld_quad = tid & 7;
     const float* qa = qsrc + static_cast<int64_t>(i0 + ld_row) * D + 4 * ld_quad;
     const float* na = nsrc + static_cast<int64_t>(c0 + ld_row) * D + 4 * ld_quad;
-    const int qa_rows = p.nqb - i0 - ld_row, na_rows = p.lsize[l] - c0 - ld_row;
+    const int qa_rows = i_end - i0 - ld_row, na_rows = p.lsize[l] - c0 - ld_row;
     const uint32_t st_off = smem_u32(ssm) + (ld_row * kScPitch + 4 * ld_quad) * 4;
 
     auto stage = [&](int kc, int s) {
@@ -139,11 +140,12 @@ __global__ void __launch_bounds__(kScThreads, 2) score_kernel(const SelectParams
         __syncthreads();  // the stage is refilled next trip
     }
 
+    const int64_t prow0 = (static_cast<int64_t>(b) * p.Hsel + hs) * p.qc - p.i_lo;  // plane row of query block 0
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         const int i = i0 + tr + 16 * m;
-        if (i >= p.nqb) continue;
-        float* dst = p.scores + (qrow0 + i) * p.total_nodes + p.loff[l];
+        if (i >= i_end) continue;
+        float* dst = p.scores + (prow0 + i) * p.total_nodes + p.loff[l];
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
             const int c = c0 + tc + 16 * n;
@@ -158,14 +160,15 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
     constexpr int DL = D / 32;  // query-summary dims per lane
     constexpr uint32_t FULL = 0xFFFFFFFFu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kDescWarps + warp;
-    if (row >= rows) return;
+    const int64_t prow = static_cast<int64_t>(blockIdx.x) * kDescWarps + warp;  // row of the chunk's plane
+    if (prow >= rows) return;
     int32_t* kl = dsm + warp * (32 * J + PISA_MAX_LEVELS);          // kept nodes of the current level
     float* pscore = reinterpret_cast<float*>(kl + 32 * J);           // straddling-node score per level
 
-    const int i = static_cast<int>(row % p.nqb);
-    const int hs = static_cast<int>((row / p.nqb) % p.Hsel);
-    const int b = static_cast<int>(row / (static_cast<int64_t>(p.nqb) * p.Hsel));
+    const int i = p.i_lo + static_cast<int>(prow % p.nqc);
+    const int hs = static_cast<int>((prow / p.nqc) % p.Hsel);
+    const int b = static_cast<int>(prow / (static_cast<int64_t>(p.nqc) * p.Hsel));
+    const int64_t row = (static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i;  // selection row
     const int kvh = hs / p.gsel_div;
     const int64_t last = p.causal ? i : p.n0_valid - 1;
     int32_t* dst = p.idx + row * p.topk;
@@ -204,7 +207,7 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
         __syncwarp();
     }
 
-    const float* srow = p.scores + row * p.total_nodes;
+    const float* srow = p.scores + ((static_cast<int64_t>(b) * p.Hsel + hs) * p.qc + (i - p.i_lo)) * p.total_nodes;
     const uint32_t lt_mask = (1u << lane) - 1u;
     // forced blocks (sink, local): not candidates at level 0, added to the output at the end
     int32_t f0, f1;
@@ -351,34 +354,40 @@ static bool launch_descent(const SelectParams& p, int64_t rows, cudaStream_t st)
 
 int dense_select_cap(int cap) { return cap <= 32 * 8 ? 256 : cap <= 32 * 16 ? 512 : cap <= 32 * 32 ? 1024 : 0; }
 
-bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st) {
-    int tiles = 0;
-    for (int l = 0; l < p.L; ++l) {
-        p.tile_off[l] = tiles;
-        p.tiles_c[l] = (p.lsize[l] + kScTile - 1) / kScTile;
-        tiles += ((p.nqb + kScTile - 1) / kScTile) * p.tiles_c[l];
-    }
-    p.tile_off[p.L] = tiles;
+bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st, int32_t* launches) {
     const size_t smem = 2 * kScStageFloats * sizeof(float);
-    dim3 grid(tiles, p.Hsel, batch);
-    if (p.D == 64) {
-        cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        score_kernel<64><<<grid, kScThreads, smem, st>>>(p);
-    } else {
-        cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        score_kernel<128><<<grid, kScThreads, smem, st>>>(p);
-    }
-    if (cudaGetLastError() != cudaSuccess) return false;
-    const int64_t rows = static_cast<int64_t>(batch) * p.Hsel * p.nqb;
+    if (cudaFuncSetAttribute(p.D == 64 ? score_kernel<64> : score_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return false;
     const int J = dense_select_cap(cap) / 32;
-    if (p.D == 64) {
-        if (J == 8) return launch_descent<64, 8>(p, rows, st);
-        if (J == 16) return launch_descent<64, 16>(p, rows, st);
-        return launch_descent<64, 32>(p, rows, st);
+    // query blocks in chunks of qc: each chunk is scored into the plane, then descended
+    for (p.i_lo = 0; p.i_lo < p.nqb; p.i_lo += p.qc) {
+        p.nqc = min(p.qc, p.nqb - p.i_lo);
+        int tiles = 0;
+        for (int l = 0; l < p.L; ++l) {
+            p.tile_off[l] = tiles;
+            p.tiles_c[l] = (p.lsize[l] + kScTile - 1) / kScTile;
+            tiles += ((p.nqc + kScTile - 1) / kScTile) * p.tiles_c[l];
+        }
+        p.tile_off[p.L] = tiles;
+        dim3 grid(tiles, p.Hsel, batch);
+        if (p.D == 64)
+            score_kernel<64><<<grid, kScThreads, smem, st>>>(p);
+        else
+            score_kernel<128><<<grid, kScThreads, smem, st>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return false;
+        const int64_t rows = static_cast<int64_t>(batch) * p.Hsel * p.nqc;
+        bool ok;
+        if (p.D == 64)
+            ok = J == 8 ? launch_descent<64, 8>(p, rows, st)
+                        : (J == 16 ? launch_descent<64, 16>(p, rows, st) : launch_descent<64, 32>(p, rows, st));
+        else
+            ok = J == 8 ? launch_descent<128, 8>(p, rows, st)
+                        : (J == 16 ? launch_descent<128, 16>(p, rows, st) : launch_descent<128, 32>(p, rows, st));
+        if (!ok) return false;
+        *launches += 2;
     }
-    if (J == 8) return launch_descent<128, 8>(p, rows, st);
-    if (J == 16) return launch_descent<128, 16>(p, rows, st);
-    return launch_descent<128, 32>(p, rows, st);
+    return true;
 }
 
 }  // namespace pisa

@@ -122,10 +122,12 @@ PISA_API pisa_status pisa_pyramid_size(const pisa_shape *shape, size_t *bytes);
  * pisa_sparse_attention need for this shape (one size serves all three).
  * The first 256 bytes are the device status word; zero them once when the
  * workspace is allocated (pisa_check_status clears them after each read).
- * Prefill with 16 or more query blocks also holds an fp32 score plane of
- * B * Hsel * (Nq / b) * total_nodes values (Hsel = heads_kv, or heads_q with
- * select_per_qhead), used by the selection.
- * Host only. */
+ * Prefill with 16 or more query blocks, while scoring every eligible node is
+ * cheaper than the sparse descent (up to about 1M tokens at block 128), also
+ * holds an fp32 score plane of B * Hsel * qc * total_nodes values (Hsel =
+ * heads_kv, or heads_q with select_per_qhead): the selection scores and
+ * descends qc query blocks at a time, qc a multiple of 128 chosen so the plane
+ * stays within 192 MiB (128 query blocks if even those need more). Host only. */
 PISA_API pisa_status pisa_workspace_size(const pisa_shape *shape, size_t *bytes);
 
 /* Step 1, the key pyramid ("Le pooling comme premiere reduction"): level 0 is
@@ -268,6 +270,18 @@ PISA_API pisa_status pisa_decode_attention_noalloc(const pisa_shape *shape, cons
  * library's array (PISA_OK if none) and clears it. `detail`, if not NULL,
  * receives the code locating the error. Allocates nothing. */
 PISA_API pisa_status pisa_decode_noalloc_check_status(uint32_t *detail, pisa_stream_t stream);
+
+/* Self-test of the bounded waits (no counterpart in the paper): enqueues one kernel whose single
+ * mbarrier wait can never complete (nothing arrives on the barrier and no copy or MMA is issued).
+ * The wait gives up after `limit_us` microseconds (1 .. 1,000,000), records PISA_ERR_TIMEOUT in
+ * the status word at the start of `ws` (detail 0x501) and the kernel returns, which is what any
+ * pipeline wait of the library does when its limit (2 s) runs out. Read the result with
+ * pisa_check_status. `ws`: device, 16-byte aligned, at least 256 bytes. Asynchronous on `stream`.
+ *
+ * Fault injection: when the environment variable PISA_FAULT is "launch", every call of this
+ * header that enqueues work returns PISA_ERR_CUDA after its argument checks, as if its first
+ * kernel launch had failed, and enqueues nothing. */
+PISA_API pisa_status pisa_selftest_wait_timeout(void *ws, uint32_t limit_us, pisa_stream_t stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace status word since the last call (PISA_OK if none) and clears it.

@@ -207,3 +207,35 @@ def test_append_pyramid_argument_checks():
     assert f.pisa_append_pyramid(ctypes.byref(s), FAKE, MISALIGNED, 0, None) == pisa.ERR_INVALID_ARG
     for old in (-64, 4096 + 64, 32):  # negative, past seq_kv, not a whole block
         assert f.pisa_append_pyramid(ctypes.byref(s), FAKE, FAKE, old, None) == pisa.ERR_INVALID_ARG
+
+
+def test_workspace_grows_no_faster_than_n_log_n():
+    """The selection's score plane is scored and descended in chunks of query blocks, so the
+    workspace of a causal prefill grows like the pyramid, the query summaries and the index rows
+    (O(N)), not like nQB x total nodes (O(N^2)): the 1M-token workload stays within a few hundred MB,
+    and from 128K to 1M to 4M tokens the growth stays within N log N."""
+    import math
+    shapes = {n: pisa.Shape(1, 8, 8, n, n, 128, 128, 8, 128, causal=1) for n in (1 << 17, 1 << 20, 1 << 22)}
+    ws = {n: pisa.workspace_size(s) for n, s in shapes.items()}
+    assert ws[1 << 20] < 400e6, ws[1 << 20]
+    ns = sorted(ws)
+    for a, b in zip(ns, ns[1:]):
+        assert ws[b] / ws[a] <= (b * math.log(b)) / (a * math.log(a)), (a, b, ws[a], ws[b])
+    # the bench workload too (GQA, 64-key blocks)
+    assert pisa.workspace_size(pisa.Shape(1, 32, 8, 1 << 17, 1 << 17, 128, 64, 4, 64, causal=1)) < 256e6
+
+
+def test_injected_launch_failure_after_argument_checks(monkeypatch):
+    """With PISA_FAULT=launch the enqueuing calls still report argument errors first; the
+    self-test's arguments are checked on the host too. (The injected PISA_ERR_CUDA itself, and
+    that nothing is enqueued, are checked on a GPU.)"""
+    monkeypatch.setenv("PISA_FAULT", "launch")
+    fake = ctypes.c_void_p(1 << 20)
+    bad = pisa.Shape(1, 3, 2, 4096, 4096, 64, 64, 4, 8)      # heads_q not a multiple of heads_kv
+    assert pisa._lib.pisa_build_pyramid(ctypes.byref(bad.c()), fake, fake, None) == pisa.ERR_INVALID_ARG
+    good = pisa.Shape(1, 2, 2, 4096, 4096, 64, 64, 4, 8)
+    assert pisa._lib.pisa_build_pyramid(ctypes.byref(good.c()), fake, None, None) == pisa.ERR_INVALID_ARG
+    assert pisa._lib.pisa_build_pyramid(ctypes.byref(good.c()), fake, fake, None) == pisa.ERR_CUDA
+    assert pisa._lib.pisa_selftest_wait_timeout(fake, 0, None) == pisa.ERR_INVALID_ARG
+    assert pisa._lib.pisa_selftest_wait_timeout(None, 10, None) == pisa.ERR_INVALID_ARG
+    assert pisa._lib.pisa_selftest_wait_timeout(fake, 10, None) == pisa.ERR_CUDA

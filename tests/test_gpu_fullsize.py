@@ -38,7 +38,7 @@ def _run(w, device):
     return shape, pyr, idx.cpu().numpy(), o, lse
 
 
-def _check_planes(w, shape, pyr, idx, o, lse, planes, n_sel, n_att, seed):
+def _check_planes(w, shape, pyr, idx, o, lse, planes, n_sel, n_att, seed, extra_blocks=()):
     """Pyramid, selection and attention of sampled (batch, KV head) planes against the oracle."""
     import block_sparse_long_pisa_b200 as pisa
     _, offs = pisa.level_layout(shape)
@@ -59,7 +59,7 @@ def _check_planes(w, shape, pyr, idx, o, lse, planes, n_sel, n_att, seed):
         else:
             extra = [i for (i, _) in workloads.needles(w, b, kvh)] if w.keys == "needle" else []
             picks = rng.choice(nqb, size=min(n_sel, nqb), replace=False).tolist()
-            blocks_sel = sorted(set(picks) | {0, nqb - 1} | set(extra))
+            blocks_sel = sorted(set(picks) | {0, nqb - 1} | set(extra) | set(extra_blocks))
         for i in blocks_sel:
             last = i if (w.causal and not w.decode) else w.n_blocks - 1
             r = oracle.select_blocks(qbar[i], levels, w.factor, w.topk, last)
@@ -98,7 +98,9 @@ def test_causal32k(cuda_device):
 def test_gqa128k_bench_configuration(cuda_device):
     w = workloads.WORKLOADS["gqa128k"]
     shape, pyr, idx, o, lse = _run(w, cuda_device)
-    _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (0, 5)], 16, 6, 2)
+    # the selection scores and descends 512 query blocks at a time: rows on both sides of each seam
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 0), (0, 5)], 16, 6, 2,
+                  extra_blocks=(511, 512, 1023, 1024, 1535, 1536))
     # every planted needle block is selected for its target query block, in every KV head
     for kvh in range(w.heads_kv):
         for (i, j) in workloads.needles(w, 0, kvh):
@@ -108,7 +110,8 @@ def test_gqa128k_bench_configuration(cuda_device):
 def test_long1m(cuda_device):
     w = workloads.WORKLOADS["long1m"]
     shape, pyr, idx, o, lse = _run(w, cuda_device)
-    _check_planes(w, shape, pyr, idx, o, lse, [(0, 3)], 12, 4, 3)
+    # 64 chunks of 128 query blocks
+    _check_planes(w, shape, pyr, idx, o, lse, [(0, 3)], 12, 4, 3, extra_blocks=(127, 128, 4095, 4096))
 
 
 def test_decode128k(cuda_device):

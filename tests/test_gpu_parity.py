@@ -372,3 +372,32 @@ def test_decode_with_spare_capacity(forced, cuda_device):
     o, lse = gu.host_f32(o), gu.host_f32(lse)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
     gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"], "spare capacity")
+
+
+@pytest.mark.parametrize("name,units", [("gqa4-d64-noncausal", 3), ("gqa4-causal-ragged", 8), ("decode-gqa4", 4)])
+def test_session_pipelined_host_forward(name, units, cuda_device):
+    """Session.forward with pinned host buffers splits the (batch, KV head) planes into ranges and
+    overlaps their copies with the computation of other ranges: prefill results equal one
+    pisa_forward on the whole device tensors bit for bit; decode (whose split count depends on the
+    rows per call) matches the oracle on the device call's selection."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL[name]
+    shape = pisa.Shape.of(w)
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    o_ref, _, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    pisa.raise_on_device_error(ws)
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    sess = pisa.Session(shape, cuda_device, units=units)
+    assert len(sess.ranges) == min(units, w.batch * w.heads_kv)
+    for _ in range(2):
+        out = sess.forward(hq, hk, hv)
+        torch.cuda.synchronize()
+        pisa.raise_on_device_error(sess.unit_ws)
+        if w.decode:
+            Q, K, V = (gu.host_f32(x) for x in (q, k, v))
+            ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, idx_override=idx.cpu().numpy())
+            gu.assert_output_close(out.float().numpy(), ref["O"], what=name)
+        else:
+            assert torch.equal(out, o_ref.cpu()), name
