@@ -212,5 +212,9 @@ bool bwd_dq_tc_supported(const BwdParams& p);
 bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
+// 2-D TMA view [rows, D] of an fp32 tensor, boxes of 32 columns x 128 rows, 128-byte swizzle.
+bool make_tmap_2d_f32(CUtensorMap* m, const void* ptr, int64_t rows, int D);
+// Dense prefill scoring of one chunk on the tensor cores (grid: tiles, Hsel, batch).
+bool launch_score_tc(const SelectParams& p, dim3 grid, cudaStream_t st);
 
 }  // namespace pisa

@@ -1,0 +1,239 @@
+// Dense prefill scoring on the tensor cores ("La selection top-K guidee par la
+// pyramide", PISA page): every query-block summary of one selection row
+// against every eligible pyramid node of the levels the descent can visit, as
+// fp32 dot products q . node, written to the score plane that descent_kernel
+// reads (same tiling, same plane, same eligibility rule as the FFMA tiles).
+//
+// One CTA per 128 query blocks x 128 nodes. The fp32 operands reach shared
+// memory by 2-D TMA (32 columns x 128 rows per box, 128-byte swizzle), D in
+// chunks of 32 through one stage per CTA; three CTAs share an SM, so one
+// CTA's copies overlap the others' splitting, MMAs and stores. Each value is split there into a tf32
+// head (its top 19 bits) and an exact fp32 remainder, and tcgen05 MMAs of kind
+// tf32 accumulate head*head + head*rest + rest*head in TMEM. The dropped
+// rest*rest term and the remainders' own tf32 rounding are below 2^-21 of
+// |q||node| per product, the size of fp32 rounding over the dot product, so
+// the ranking the descent draws from these scores differs from an fp32 dot
+// product only where two scores agree to about six digits (a near-tie).
+//
+// Roles: thread 0 issues the copies and the MMAs, all 256 threads split the
+// operands, and the eight warps read the 128 x 128 accumulator out of TMEM
+// (warp w: query blocks 32 (w % 4).., nodes 64 (w / 4)..) and store it through a
+// padded shared tile, 32 consecutive nodes of one row per store instruction.
+#include <cuda.h>
+
+#include "pisa_device.cuh"
+
+namespace pisa {
+
+constexpr int kStTile = 128;                 // query blocks and nodes per tile
+constexpr int kStChunk = 32;                 // D per stage (one 128-byte swizzle atom of fp32)
+constexpr int kStThreads = 256;
+constexpr int kStOp = kStTile * kStChunk * 4;  // one operand chunk: 16 KB
+constexpr int kStStage = 4 * kStOp;            // A head, A rest, B head, B rest
+constexpr int kStStages = 1;                   // one stage: three CTAs share an SM and overlap
+constexpr int kStSmem = 1024 + kStStages * kStStage + 256;
+
+// kind::tf32 instruction descriptor: fp32 accumulator, A and B tf32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int m, int n) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Splits one loaded operand chunk in place: head = x with its 13 low mantissa bits cleared (exact
+// in tf32), rest = x - head (exact in fp32), written at the same swizzled offsets.
+__device__ __forceinline__ void split_chunk(uint8_t* head, uint8_t* rest, int tid) {
+    float4* h4 = reinterpret_cast<float4*>(head);
+    float4* r4 = reinterpret_cast<float4*>(rest);
+#pragma unroll 4
+    for (int e = tid; e < kStOp / 16; e += kStThreads) {
+        const float4 x = h4[e];
+        float4 h, r;
+        h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+        h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+        h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+        h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+        r.x = x.x - h.x;
+        r.y = x.y - h.y;
+        r.z = x.z - h.z;
+        r.w = x.w - h.w;
+        h4[e] = h;
+        r4[e] = r;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kStThreads, 3)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmN,
+                    const SelectParams p) {
+    constexpr int NC = D / kStChunk;
+    extern __shared__ uint8_t st_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(st_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kStStages * kStStage);  // per stage
+    uint64_t* done = full + kStStages;                                          // per stage: its MMAs completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + kStStages);
+
+    const int hs = blockIdx.y, b = blockIdx.z;
+    int tile = blockIdx.x, l = 0;
+    while (l + 1 < p.L && tile >= p.tile_off[l + 1]) ++l;
+    tile -= p.tile_off[l];
+    const int i_end = p.i_lo + p.nqc;
+    const int i0 = p.i_lo + (tile / p.tiles_c[l]) * kStTile;
+    const int c0 = (tile % p.tiles_c[l]) * kStTile;
+    const int i_hi = min(i0 + kStTile, i_end) - 1;
+    const int64_t last_hi = p.causal ? i_hi : p.n0_valid - 1;
+    // the descent's start level and the eligible nodes only grow with the query block
+    int start = -1;
+    for (int ll = p.L - 1; ll >= 0; --ll)
+        if (last_hi / p.width[ll] + 1 > p.budget[ll]) {
+            start = ll;
+            break;
+        }
+    if (start < l || c0 > last_hi / p.width[l]) return;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kvh = hs / p.gsel_div;
+    const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i0);
+    const int nrow = static_cast<int>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.total_nodes + p.loff[l] + c0);
+    const uint32_t detail_base = kKernSelect << 8;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(done + s, 1);
+        }
+        fence_barrier_init();
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmN);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    auto stage_ptr = [&](int s, int op) { return base + s * kStStage + op * kStOp; };  // op: 0 Ah 1 Ar 2 Bh 3 Br
+    auto load = [&](int c) {
+        const int s = c % kStStages;
+        mbar_arrive_expect_tx(full + s, 2 * kStOp);
+        tma_load_2d(stage_ptr(s, 0), &tmQ, c * kStChunk, qrow, full + s);
+        tma_load_2d(stage_ptr(s, 2), &tmN, c * kStChunk, nrow, full + s);
+    };
+    int loaded = 0;        // thread 0: chunks whose copies were started
+    int last_commit = -1;  // thread 0: last chunk whose MMAs were issued
+    if (tid == 0)
+        for (; loaded < kStStages && loaded < NC; ++loaded) load(loaded);
+
+    bool ok = true;
+    constexpr uint32_t idesc = idesc_tf32_f32(128, 128);
+    for (int c = 0; c < NC; ++c) {
+        const int s = c % kStStages, use = c / kStStages;
+        if (ok) ok = mbar_wait(full + s, use & 1, p.status, detail_base | 0x41u);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        split_chunk(stage_ptr(s, 0), stage_ptr(s, 1), tid);
+        split_chunk(stage_ptr(s, 2), stage_ptr(s, 3), tid);
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t ah = smem_desc_sw128(smem_u32(stage_ptr(s, 0)), 16, 1024);
+            const uint64_t ar = smem_desc_sw128(smem_u32(stage_ptr(s, 1)), 16, 1024);
+            const uint64_t bh = smem_desc_sw128(smem_u32(stage_ptr(s, 2)), 16, 1024);
+            const uint64_t br = smem_desc_sw128(smem_u32(stage_ptr(s, 3)), 16, 1024);
+#pragma unroll
+            for (int ks = 0; ks < kStChunk / 8; ++ks) {
+                const uint32_t off = static_cast<uint32_t>((ks * 32) >> 4);  // 8 tf32 = 32 bytes per K step
+                mma_tf32_ss(tm, ah + off, bh + off, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+                mma_tf32_ss(tm, ah + off, br + off, idesc, 1u);
+                mma_tf32_ss(tm, ar + off, bh + off, idesc, 1u);
+            }
+            mma_commit(done + s);
+            last_commit = c;
+            if (c + kStStages < NC) {
+                // the stage is refilled once its MMAs have read it
+                if (mbar_wait(done + s, use & 1, p.status, detail_base | 0x42u)) {
+                    load(c + kStStages);
+                    ++loaded;
+                } else {
+                    ok = false;
+                }
+            }
+        }
+    }
+    // every MMA issued has completed, and every copy started has landed, before the epilogue and
+    // before shared and tensor memory are released
+    if (tid == 0) {
+        // the last commit covers every MMA issued before it; the last two copies are the only ones
+        // that can still be in flight (their phases are the latest of their barriers)
+        if (last_commit >= 0)
+            mbar_wait(done + last_commit % kStStages, (last_commit / kStStages) & 1, p.status, detail_base | 0x43u);
+        for (int c = max(0, loaded - kStStages); c < loaded; ++c)
+            mbar_wait(full + c % kStStages, (c / kStStages) & 1, p.status, detail_base | 0x44u);
+    }
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
+    if (ok) {
+        // warp w reads TMEM lanes 32 (w % 4).. (query blocks) and node columns 64 (w / 4).. in two
+        // 32-column pieces; each piece goes through a padded shared tile so that the stores cover
+        // 32 consecutive nodes of one row per instruction (the stages are free: every MMA is done)
+        float* stile = reinterpret_cast<float*>(base) + warp * 32 * 33;
+        const int q4 = warp & 3, half = warp >> 2;
+        const int ncols = min(kStTile, p.lsize[l] - c0);
+        const int64_t prow0 = (static_cast<int64_t>(b) * p.Hsel + hs) * p.qc - p.i_lo;  // plane row of block 0
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+            const int col0 = half * 64 + q * 32;
+            uint32_t v[32];
+            tmem_ld32(tm + (static_cast<uint32_t>(q4 * 32) << 16) + col0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) stile[lane * 33 + k] = __uint_as_float(v[k]);
+            __syncwarp();
+            const int col = col0 + lane;
+#pragma unroll 4
+            for (int r = 0; r < 32; ++r) {
+                const int i = i0 + q4 * 32 + r;
+                if (i < i_end && col < ncols) p.scores[(prow0 + i) * p.total_nodes + p.loff[l] + c0 + col] = stile[r * 33 + lane];
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 128);
+    }
+}
+
+bool launch_score_tc(const SelectParams& p, dim3 grid, cudaStream_t st) {
+    const int64_t qrows = static_cast<int64_t>(grid.z) * p.Hsel * p.nqb;
+    const int64_t nrows = static_cast<int64_t>(grid.z) * p.Hkv * p.total_nodes;
+    CUtensorMap tq, tn;
+    if (!make_tmap_2d_f32(&tq, p.qbar, qrows, p.D) || !make_tmap_2d_f32(&tn, p.pyr, nrows, p.D)) return false;
+    static bool configured[2] = {false, false};
+    const int k = p.D == 64 ? 0 : 1;
+    if (!configured[k]) {
+        if (cudaFuncSetAttribute(k == 0 ? score_tc_kernel<64> : score_tc_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem) != cudaSuccess)
+            return false;
+        configured[k] = true;
+    }
+    if (k == 0)
+        score_tc_kernel<64><<<grid, kStThreads, kStSmem, st>>>(tq, tn, p);
+    else
+        score_tc_kernel<128><<<grid, kStThreads, kStSmem, st>>>(tq, tn, p);
+    return cudaGetLastError() == cudaSuccess;
+}
+
+}  // namespace pisa

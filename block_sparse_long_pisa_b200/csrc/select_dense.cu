@@ -1,13 +1,12 @@
 // Pyramid-guided top-K selection for prefill ("La selection top-K guidee par la
-// pyramide", PISA page), in two kernels.
+// pyramide", PISA page), in two kernels per chunk of query blocks.
 //
-// score_kernel: every query-block summary of one selection row against every
-// eligible node of every level the descent can visit, as fp32 dot products
-// (a dense, register-tiled FP32 product: 128 query blocks x 128 nodes per CTA,
-// D in chunks of 32 staged by cp.async, each thread an 8 x 8 block of scores).
-// A query block at level l needs nodes c <= last / f^l, and only when the
-// descent starts at l or above, so tiles entirely outside that region exit at
-// once. The scores go to an fp32 plane [rows, total_nodes] in the workspace.
+// score_tc_kernel (score_tc.cu): every query-block summary of one selection
+// row against every eligible node of every level the descent can visit, as
+// fp32-accurate dot products on the tensor cores, 128 query blocks x 128 nodes
+// per CTA. A query block at level l needs nodes c <= last / f^l, and only when
+// the descent starts at l or above, so tiles entirely outside that region exit
+// at once. The scores go to an fp32 plane [rows, total_nodes] in the workspace.
 //
 // descent_kernel: one warp per query block. It walks down from the start level
 // (the coarsest whose eligible nodes outnumber its budget), reads the scores of
@@ -26,10 +25,6 @@
 namespace pisa {
 
 constexpr int kScTile = 128;      // query blocks and nodes per score tile
-constexpr int kScChunk = 32;      // D per staged chunk
-constexpr int kScPitch = 36;      // floats per staged row (keeps LDS.128 conflict-free)
-constexpr int kScThreads = 256;
-constexpr int kScStageFloats = 2 * kScTile * kScPitch;
 constexpr int kDescWarps = 8;
 
 __device__ __forceinline__ uint32_t dorder_bits(float f) {
@@ -48,110 +43,6 @@ __device__ __forceinline__ int start_level(const SelectParams& p, int64_t last) 
     for (int l = p.L - 1; l >= 0; --l)
         if (last / p.width[l] + 1 > p.budget[l]) return l;
     return -1;
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-template <int D>
-__global__ void __launch_bounds__(kScThreads, 2) score_kernel(const SelectParams p) {
-    extern __shared__ __align__(16) float ssm[];
-    const int hs = blockIdx.y, b = blockIdx.z;
-    int tile = blockIdx.x, l = 0;
-    while (l + 1 < p.L && tile >= p.tile_off[l + 1]) ++l;
-    tile -= p.tile_off[l];
-    const int i_end = p.i_lo + p.nqc;  // this chunk's query blocks: [i_lo, i_end)
-    const int i0 = p.i_lo + (tile / p.tiles_c[l]) * kScTile;
-    const int c0 = (tile % p.tiles_c[l]) * kScTile;
-    const int i_hi = min(i0 + kScTile, i_end) - 1;
-    const int64_t last_hi = p.causal ? i_hi : p.n0_valid - 1;
-    // the start level and the eligible range only grow with the query block
-    if (start_level(p, last_hi) < l || c0 > last_hi / p.width[l]) return;
-
-    const int kvh = hs / p.gsel_div;
-    const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb;
-    const float* qsrc = p.qbar + qrow0 * D;
-    const float* nsrc = p.pyr + ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.total_nodes + p.loff[l]) * D;
-    const int tid = threadIdx.x;
-    // staging: thread copies 16 bytes of rows ld_row + 32 r of both operands
-    const int ld_row = tid >> 3, ld_quad = tid & 7;
-    const float* qa = qsrc + static_cast<int64_t>(i0 + ld_row) * D + 4 * ld_quad;
-    const float* na = nsrc + static_cast<int64_t>(c0 + ld_row) * D + 4 * ld_quad;
-    const int qa_rows = i_end - i0 - ld_row, na_rows = p.lsize[l] - c0 - ld_row;
-    const uint32_t st_off = smem_u32(ssm) + (ld_row * kScPitch + 4 * ld_quad) * 4;
-
-    auto stage = [&](int kc, int s) {
-        const uint32_t sa = st_off + s * kScStageFloats * 4, sb = sa + kScTile * kScPitch * 4;
-#pragma unroll
-        for (int r = 0; r < kScTile / 32; ++r) {
-            const bool va = 32 * r < qa_rows, vb = 32 * r < na_rows;
-            cp_async16(sa + r * 32 * kScPitch * 4, va ? qa + r * 32 * D + kc * kScChunk : qsrc, va);
-            cp_async16(sb + r * 32 * kScPitch * 4, vb ? na + r * 32 * D + kc * kScChunk : nsrc, vb);
-        }
-        cp_async_commit();
-    };
-
-    // thread (tr, tc) owns query blocks tr + 16 m and nodes tc + 16 n
-    const int warp = tid >> 5, lane = tid & 31;
-    const int tr = 2 * warp + (lane >> 4), tc = lane & 15;
-    float acc[8][8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int n = 0; n < 8; ++n) acc[m][n] = 0.f;
-
-    constexpr int NK = D / kScChunk;
-    stage(0, 0);
-#pragma unroll 1
-    for (int kc = 0; kc < NK; ++kc) {
-        if (kc + 1 < NK) {
-            stage(kc + 1, (kc + 1) & 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const float* As = ssm + (kc & 1) * kScStageFloats;
-        const float* Bs = As + kScTile * kScPitch;
-#pragma unroll
-        for (int dq = 0; dq < kScChunk / 4; ++dq) {
-            float4 bv[8];
-#pragma unroll
-            for (int n = 0; n < 8; ++n) bv[n] = *reinterpret_cast<const float4*>(Bs + (tc + 16 * n) * kScPitch + 4 * dq);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float4 a = *reinterpret_cast<const float4*>(As + (tr + 16 * m) * kScPitch + 4 * dq);
-#pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    float s = acc[m][n];
-                    s = fmaf(a.x, bv[n].x, s);
-                    s = fmaf(a.y, bv[n].y, s);
-                    s = fmaf(a.z, bv[n].z, s);
-                    s = fmaf(a.w, bv[n].w, s);
-                    acc[m][n] = s;
-                }
-            }
-        }
-        __syncthreads();  // the stage is refilled next trip
-    }
-
-    const int64_t prow0 = (static_cast<int64_t>(b) * p.Hsel + hs) * p.qc - p.i_lo;  // plane row of query block 0
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int i = i0 + tr + 16 * m;
-        if (i >= i_end) continue;
-        float* dst = p.scores + (prow0 + i) * p.total_nodes + p.loff[l];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int c = c0 + tc + 16 * n;
-            if (c < p.lsize[l]) dst[c] = acc[m][n];
-        }
-    }
 }
 
 template <int D, int J>
@@ -355,10 +246,6 @@ static bool launch_descent(const SelectParams& p, int64_t rows, cudaStream_t st)
 int dense_select_cap(int cap) { return cap <= 32 * 8 ? 256 : cap <= 32 * 16 ? 512 : cap <= 32 * 32 ? 1024 : 0; }
 
 bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st, int32_t* launches) {
-    const size_t smem = 2 * kScStageFloats * sizeof(float);
-    if (cudaFuncSetAttribute(p.D == 64 ? score_kernel<64> : score_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-        return false;
     const int J = dense_select_cap(cap) / 32;
     // query blocks in chunks of qc: each chunk is scored into the plane, then descended
     for (p.i_lo = 0; p.i_lo < p.nqb; p.i_lo += p.qc) {
@@ -371,11 +258,7 @@ bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st
         }
         p.tile_off[p.L] = tiles;
         dim3 grid(tiles, p.Hsel, batch);
-        if (p.D == 64)
-            score_kernel<64><<<grid, kScThreads, smem, st>>>(p);
-        else
-            score_kernel<128><<<grid, kScThreads, smem, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return false;
+        if (!launch_score_tc(p, grid, st)) return false;
         const int64_t rows = static_cast<int64_t>(batch) * p.Hsel * p.nqc;
         bool ok;
         if (p.D == 64)
