@@ -82,19 +82,6 @@ struct PrefillCfg {
     static_assert(SMEM < (1 << 18), "descriptor offsets assume shared addresses below 2^18");
 };
 
-// First pass: every row keeps the maximum of its first key group as the
-// reference for all later groups, so the two warps of a row need not agree on
-// a new maximum per group. Probabilities then stay below 2^kFirstPassLimit;
-// a row whose scores exceed that (in log2 units) marks the CTA, which redoes
-// its unit in a second pass with the exact lazy rescale below.
-constexpr float kFirstPassLimit = 16.0f;
-// Second pass: the running max is kept until a new row max exceeds it by this
-// much (log2 units), so probabilities stay below 2^8.
-constexpr float kRescaleThreshold = 8.0f;
-// Named barrier at which all roles learn whether a second pass runs (1..8
-// are the softmax warp pairs' barriers).
-constexpr uint32_t kPassBarrier = 15;
-
 template <int D, int BLK, int NM>
 __global__ void __launch_bounds__(PrefillCfg<D, BLK, NM>::THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -639,6 +626,12 @@ pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, co
         return PISA_ERR_CUDA;
     const int nm = p.gh * pl.blk > 128 ? 2 : 1;
     dim3 grid(pl.nqb, pl.Hsel * p.chunks, pl.B);
+    if (nm == 1 && pl.nqb >= 2) {
+        // units of at most 128 rows: two query blocks per CTA, one per tile
+        if (!launch_attn_prefill_dual(pl.D, pl.blk, tq, tk, tv, p, grid, st)) return PISA_ERR_CUDA;
+        ++*launches;
+        return PISA_OK;
+    }
     bool ok = false;
     if (pl.D == 128 && pl.blk == 64)
         ok = nm == 2 ? launch_variant<128, 64, 2>(tq, tk, tv, p, grid, st)

@@ -16,6 +16,19 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // Suspend-time hint of one mbarrier wait attempt (ns); the bound above still applies.
 constexpr uint32_t kTryWaitHintNs = 1000000u;
 
+// First pass: every row keeps the maximum of its first key group as the
+// reference for all later groups, so the two warps of a row need not agree on
+// a new maximum per group. Probabilities then stay below 2^kFirstPassLimit;
+// a row whose scores exceed that (in log2 units) marks the CTA, which redoes
+// its unit in a second pass with the exact lazy rescale below.
+constexpr float kFirstPassLimit = 16.0f;
+// Second pass: the running max is kept until a new row max exceeds it by this
+// much (log2 units), so probabilities stay below 2^8.
+constexpr float kRescaleThreshold = 8.0f;
+// Named barrier at which all roles learn whether a second pass runs (1..8
+// are the softmax warp pairs' barriers).
+constexpr uint32_t kPassBarrier = 15;
+
 // Selected blocks per query block the prefill attention kernel holds on chip.
 constexpr int kMaxPrefillTopk = 256;
 // Largest number of selected blocks one decode CTA streams (its block list lives in shared memory).
@@ -201,6 +214,10 @@ bool launch_select_dense(SelectParams p, int32_t batch, int cap, cudaStream_t st
 // Prefill attention: builds the tensor maps and picks the kernel variant.
 pisa_status launch_attn_prefill(const Plan& pl, const void* Q, const void* K, const void* V, const AttnParams& p,
                                 cudaStream_t st, int32_t* launches);
+// Prefill attention with two units (neighbouring query blocks) per CTA, one per tensor-core tile,
+// for units of at most 128 rows; grid as for one unit per CTA (x = query blocks).
+bool launch_attn_prefill_dual(int D, int blk, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                              const AttnParams& p, dim3 grid, cudaStream_t st);
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
 bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
 // Backward column pass on the tensor cores (head dim 128, 64-key blocks); false when the shape is
