@@ -264,6 +264,7 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
         sp.width[l] = w;
         w = w > (int64_t(1) << 40) ? w : w * pl.f;
     }
+    sp.fshift = (pl.f & (pl.f - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(pl.f)) : -1;
     sp.scores = pl.dense_select ? reinterpret_cast<float*>(ws + pl.ws_scores) : nullptr;
     sp.qc = pl.dense_qc;
     if (!launch_select(sp, pl.B, st, &g_launches)) return PISA_ERR_CUDA;

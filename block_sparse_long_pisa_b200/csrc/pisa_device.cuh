@@ -287,6 +287,22 @@ __device__ __forceinline__ int forced_blocks(int32_t mask, int32_t local, int32_
     return n < cap ? n : cap;
 }
 
+// ---------------------------------------------------------------- selection index arithmetic
+
+// x / f^l (x >= 0): a shift when the pooling factor is a power of two, else a 64-bit division.
+__device__ __forceinline__ int64_t div_width(const SelectParams& p, int64_t x, int l) {
+    if (p.fshift >= 0) {
+        const int s = p.fshift * l;
+        return s >= 63 ? 0 : (x >> s);
+    }
+    return x / p.width[l];
+}
+
+// t / f for t >= 0 (a child's position among the candidates -> its parent's slot).
+__device__ __forceinline__ int div_factor(const SelectParams& p, int t) {
+    return p.fshift >= 0 ? (t >> p.fshift) : t / p.factor;
+}
+
 // ---------------------------------------------------------------- small math
 
 __device__ __forceinline__ float fast_exp2(float x) {

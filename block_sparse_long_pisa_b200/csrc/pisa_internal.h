@@ -146,6 +146,7 @@ struct SelectParams {
     int32_t loff[PISA_MAX_LEVELS];
     int32_t budget[PISA_MAX_LEVELS];
     int64_t width[PISA_MAX_LEVELS];  // f^l (saturated)
+    int32_t fshift;                  // log2 f when f is a power of two, else -1
     float* scores;                   // dense prefill scoring: fp32 [B, Hsel, qc, total_nodes], or null
     int32_t qc;                      // query blocks per dense chunk (plane rows per selection row)
     int32_t i_lo, nqc;               // the chunk being scored: query blocks [i_lo, i_lo + nqc)

@@ -94,11 +94,11 @@ __global__ void __launch_bounds__(kStThreads, 3)
     // the descent's start level and the eligible nodes only grow with the query block
     int start = -1;
     for (int ll = p.L - 1; ll >= 0; --ll)
-        if (last_hi / p.width[ll] + 1 > p.budget[ll]) {
+        if (div_width(p, last_hi, ll) + 1 > p.budget[ll]) {
             start = ll;
             break;
         }
-    if (start < l || c0 > last_hi / p.width[l]) return;
+    if (start < l || c0 > div_width(p, last_hi, l)) return;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kvh = hs / p.gsel_div;

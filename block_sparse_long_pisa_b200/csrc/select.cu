@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
         float sum = plane[static_cast<int64_t>(p.loff[0] + last) * D + d];
         for (int l = 1; l < p.L; ++l) {
             const int64_t wl = p.width[l], wb = p.width[l - 1];
-            const int64_t c_l = last / wl, c_b = last / wb;
+            const int64_t c_l = div_width(p, last, l), c_b = div_width(p, last, l - 1);
             // at most f-1 full children precede the straddling one; load them together
             float ch[8];
             const int nch = static_cast<int>(c_b - c_l * p.factor);
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     // coarsest level whose eligible nodes exceed its budget
     int l0 = -1;
     for (int l = p.L - 1; l >= 0; --l) {
-        if (last / p.width[l] + 1 > p.budget[l]) {
+        if (div_width(p, last, l) + 1 > p.budget[l]) {
             l0 = l;
             break;
         }
@@ -124,14 +124,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
         const int nkeep = last + 1;
         for (int t = tid; t < p.topk; t += kSelThreads) dst[t] = t < nkeep ? t : -1;
     } else {
-        int ncand = static_cast<int>(last / p.width[l0] + 1);
+        int ncand = static_cast<int>(div_width(p, last, l0) + 1);
         // at level 0 the forced blocks (all eligible) are not candidates
         for (int t = tid; t < ncand; t += kSelThreads) cand[t] = (l0 == 0 && (t == f0 || t == f1)) ? -1 : t;
         if (tid == 0) s_nvalid = l0 == 0 ? ncand - nf : ncand;
         __syncthreads();
         for (int l = l0; l >= 0; --l) {
             const int n = next_pow2(ncand);
-            const int64_t c_part = last / p.width[l];
+            const int64_t c_part = div_width(p, last, l);
             const bool has_part = min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
             // 8 lanes per candidate: each warp load instruction covers four whole 128-byte lines;
             // each group issues the loads of kSelBatch candidates before any arithmetic
@@ -244,15 +244,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
             const int nkeep = s_scan[0];
             if (l > 0) {
                 // the next candidates: children of the kept parents, parents ascending
-                const int64_t last_below = last / p.width[l - 1];
+                const int64_t last_below = div_width(p, last, l - 1);
                 const int n_below = p.lsize[l - 1];
                 const int slots = nkeep * p.factor;
                 if (tid == 0) s_nvalid = 0;
                 __syncthreads();
                 int valid_here = 0;
                 for (int t = tid; t < slots; t += kSelThreads) {
-                    const int32_t c = kept[t / p.factor];
-                    const int64_t ch = static_cast<int64_t>(c) * p.factor + (t % p.factor);
+                    const int r = div_factor(p, t);
+                    const int32_t c = kept[r];
+                    const int64_t ch = static_cast<int64_t>(c) * p.factor + (t - r * p.factor);
                     const bool ok = ch <= last_below && ch < n_below && (l > 1 || (ch != f0 && ch != f1));
                     cand[t] = ok ? static_cast<int32_t>(ch) : -1;
                     valid_here += ok;

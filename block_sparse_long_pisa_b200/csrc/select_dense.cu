@@ -41,7 +41,7 @@ __device__ __forceinline__ float dorder_bits_inv(uint32_t e) {
 // eligible block fits the level-0 budget.
 __device__ __forceinline__ int start_level(const SelectParams& p, int64_t last) {
     for (int l = p.L - 1; l >= 0; --l)
-        if (last / p.width[l] + 1 > p.budget[l]) return l;
+        if (div_width(p, last, l) + 1 > p.budget[l]) return l;
     return -1;
 }
 
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
         }
         for (int l = 1; l <= l0; ++l) {
             const int64_t wl = p.width[l], wb = p.width[l - 1];
-            const int64_t c_l = last / wl, c_b = last / wb;
+            const int64_t c_l = div_width(p, last, l), c_b = div_width(p, last, l - 1);
             for (int64_t c = c_l * p.factor; c < c_b; ++c) {
                 const float* v = plane + (p.loff[l - 1] + c) * D + lane * DL;
 #pragma unroll
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
     float margin = __int_as_float(0x7F800000);
     int32_t node[J];
     {
-        const int64_t cnt0 = last / p.width[l0] + 1;
+        const int64_t cnt0 = div_width(p, last, l0) + 1;
 #pragma unroll
         for (int j = 0; j < J; ++j) node[j] = 32 * j + lane < cnt0 ? 32 * j + lane : -1;
     }
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
             for (int j = 0; j < J; ++j)
                 if (node[j] == f0 || node[j] == f1) node[j] = -1;
         }
-        const int64_t c_part = last / p.width[l];
+        const int64_t c_part = div_width(p, last, l);
         const bool has_part = min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
         const float ps = has_part ? pscore[l] : 0.f;
         uint32_t hi[J];
@@ -218,12 +218,12 @@ __global__ void __launch_bounds__(32 * kDescWarps) descent_kernel(const SelectPa
             if (p.margin != nullptr && lane == 0) p.margin[row] = margin;
             return;
         }
-        const int64_t last_below = last / p.width[l - 1];
+        const int64_t last_below = div_width(p, last, l - 1);
         const int n_below = p.lsize[l - 1];
 #pragma unroll
         for (int j = 0; j < J; ++j) {
             const int t = 32 * j + lane;
-            const int r = t / p.factor;
+            const int r = div_factor(p, t);
             int32_t ch = -1;
             if (r < nkeep) {
                 const int64_t c = static_cast<int64_t>(kl[r]) * p.factor + (t - r * p.factor);
