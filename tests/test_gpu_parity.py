@@ -401,3 +401,31 @@ def test_session_pipelined_host_forward(name, units, cuda_device):
             gu.assert_output_close(out.float().numpy(), ref["O"], what=name)
         else:
             assert torch.equal(out, o_ref.cpu()), name
+
+
+@pytest.mark.parametrize("name", ["gqa4-d64-noncausal", "gqa4-causal-ragged"])
+def test_units_shard_without_changing_results(name, cuda_device):
+    """The premise of sharding over GPUs: (batch, KV head) units are independent. A call on any
+    subset of the units (one sequence of the batch, a range of KV heads with their query heads)
+    gives exactly, bit for bit, what the call on the whole batch gives for those units, so a rank
+    that processes its shard returns the single-process output for it."""
+    import dataclasses
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w = SMALL[name]
+    if w.batch == 1:
+        w = w.replace(batch=2)
+    shape = pisa.Shape.of(w)
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    o, lse, idx = pisa.forward(shape, q, k, v, pisa.new_workspace(shape, cuda_device), idx=True)
+    g = w.heads_q // w.heads_kv
+    shards = [(b, h0, h1) for b in range(w.batch) for (h0, h1) in ((0, 1), (1, w.heads_kv))]
+    for b, h0, h1 in shards:
+        sub = dataclasses.replace(shape, batch=1, heads_q=(h1 - h0) * g, heads_kv=h1 - h0)
+        qs = q[b:b + 1, h0 * g:h1 * g].contiguous()
+        ks, vs = k[b:b + 1, h0:h1].contiguous(), v[b:b + 1, h0:h1].contiguous()
+        os_, ls, is_ = pisa.forward(sub, qs, ks, vs, pisa.new_workspace(sub, cuda_device), idx=True)
+        torch.cuda.synchronize()
+        assert torch.equal(os_, o[b:b + 1, h0 * g:h1 * g]), (name, b, h0, h1)
+        assert torch.equal(ls, lse[b:b + 1, h0 * g:h1 * g]), (name, b, h0, h1)
+        assert torch.equal(is_, idx[b:b + 1, h0:h1]), (name, b, h0, h1)
