@@ -183,7 +183,8 @@ static pisa_status pyramid_range(const Plan& pl, const void* K, float* pyr, int3
 
 // Whole pyramid: subtrees of S = f^m key blocks (f^m <= max(64, f), m <= L - 1) formed in one
 // launch, the levels above them in a second; a single-level pyramid or a factor above 64 takes
-// the per-level path. Both give the same values bit for bit.
+// the per-level path. Both give the same values bit for bit. (Subtrees of 16 blocks at the 128K
+// workload, 1024 CTAs instead of 256, measured slower: 0.068 vs 0.062 ms for the stage.)
 static pisa_status build_pyramid(const Plan& pl, const void* K, float* pyr, cudaStream_t st) {
     if (pl.L < 2 || pl.f > 64) return pyramid_range(pl, K, pyr, 0, pl.n0_cap, st);
     SubtreeParams p{};

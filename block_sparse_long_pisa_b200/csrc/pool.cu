@@ -17,7 +17,9 @@
 // (one warp per block, the block_mean_kernel arithmetic), keeps their means in
 // shared memory and forms the m levels above them inside the subtree; one CTA
 // per plane then forms the levels above the subtree roots. Compared with one
-// launch per level, the small levels no longer cost a launch each.
+// launch per level, the small levels no longer cost a launch each; the second
+// kernel is a programmatic dependent of the first (it is launched while the
+// subtrees stream and waits for their completion), so its launch is hidden.
 //
 // Every path computes a row mean and a node mean with the same device
 // functions in the same order, so a build, an append (which recomputes a
@@ -153,6 +155,9 @@ template <int D>
 __global__ void __launch_bounds__(512) pyramid_subtree_kernel(const SubtreeParams p) {
     extern __shared__ __align__(16) float tree[];
     constexpr int CH = D / 8;
+    // the top-level kernel may be launched now (it waits for this grid's completion before it
+    // reads anything), so its launch overlaps this grid's work
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t plane = blockIdx.x / p.subtrees;
     const int sub = static_cast<int>(blockIdx.x % p.subtrees);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -210,6 +215,9 @@ __global__ void __launch_bounds__(512) pyramid_subtree_kernel(const SubtreeParam
 // Levels m+1 .. L-1 of one plane per CTA, level after level, from the rows below in global memory
 // (the subtree roots, then this CTA's own output).
 __global__ void __launch_bounds__(512) pyramid_top_kernel(const SubtreeParams p) {
+    // launched as a programmatic dependent of the subtree kernel: wait until that grid has
+    // completed and its writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t plane = blockIdx.x;
     float* out_plane = p.pyr + plane * p.plane_rows * p.D;
     int64_t width_below = 1;
@@ -261,7 +269,16 @@ bool launch_pyramid_two_pass(const SubtreeParams& p, cudaStream_t st, int32_t* l
     ++*launches;
     if (cudaGetLastError() != cudaSuccess) return false;
     if (p.m + 1 < p.L) {
-        pyramid_top_kernel<<<static_cast<unsigned>(p.planes), 512, 0, st>>>(p);
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(static_cast<unsigned>(p.planes));
+        cfg.blockDim = dim3(512);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, pyramid_top_kernel, p) != cudaSuccess) return false;
         ++*launches;
     }
     return cudaGetLastError() == cudaSuccess;
