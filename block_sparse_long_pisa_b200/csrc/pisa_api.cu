@@ -116,6 +116,10 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
         const int64_t qc = chunks <= 1 ? p->nqb : ((p->nqb + chunks - 1) / chunks + 127) / 128 * 128;
         p->dense_qc = static_cast<int32_t>(qc);
         o = align256(o + static_cast<size_t>(p->B) * p->Hsel * p->dense_qc * p->total_nodes * sizeof(float));
+        p->ws_split = o;
+        o = align256(o + 2 * (static_cast<size_t>(p->B) * p->Hsel * p->nqb + static_cast<size_t>(p->B) * p->Hkv *
+                                                                               p->total_nodes) *
+                             p->D * sizeof(float));
     }
     p->ws_total = o;
     return PISA_OK;
@@ -268,6 +272,17 @@ static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, c
     sp.fshift = (pl.f & (pl.f - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(pl.f)) : -1;
     sp.scores = pl.dense_select ? reinterpret_cast<float*>(ws + pl.ws_scores) : nullptr;
     sp.qc = pl.dense_qc;
+    if (pl.dense_select) {
+        // tf32 head and remainder of the summaries and of the pyramid for the tensor-core scoring
+        const int64_t nq = static_cast<int64_t>(pl.B) * pl.Hsel * pl.nqb * pl.D;
+        const int64_t nn = static_cast<int64_t>(pl.B) * pl.Hkv * pl.total_nodes * pl.D;
+        float* qs = reinterpret_cast<float*>(ws + pl.ws_split);
+        float* ns = qs + 2 * nq;
+        if (!launch_split_tf32(qbar, qs, qs + nq, nq, pyr, ns, ns + nn, nn, st)) return PISA_ERR_CUDA;
+        ++g_launches;
+        sp.qsplit = qs;
+        sp.nsplit = ns;
+    }
     if (!launch_select(sp, pl.B, st, &g_launches)) return PISA_ERR_CUDA;
     return PISA_OK;
 }

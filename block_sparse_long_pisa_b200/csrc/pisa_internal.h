@@ -86,6 +86,7 @@ struct Plan {
     size_t ws_pyramid, ws_qbar, ws_idx, ws_part, ws_scores, ws_total;
     int32_t dense_select;       // prefill selection scores densely (score plane in the workspace)
     int32_t dense_qc;           // query blocks per dense-selection chunk (a multiple of 128, or nqb)
+    size_t ws_split;            // dense selection: tf32 head and remainder of the summaries and nodes
     size_t pyramid_bytes;
 };
 
@@ -149,6 +150,8 @@ struct SelectParams {
     int32_t fshift;                  // log2 f when f is a power of two, else -1
     float* scores;                   // dense prefill scoring: fp32 [B, Hsel, qc, total_nodes], or null
     int32_t qc;                      // query blocks per dense chunk (plane rows per selection row)
+    const float* qsplit;             // dense scoring: [2, B * Hsel * nqb, D] tf32 head, then remainder
+    const float* nsplit;             // dense scoring: [2, B * Hkv * total_nodes, D] likewise
     int32_t i_lo, nqc;               // the chunk being scored: query blocks [i_lo, i_lo + nqc)
     int32_t tile_off[PISA_MAX_LEVELS + 1];  // score tiles before level l (set by the launcher)
     int32_t tiles_c[PISA_MAX_LEVELS];       // node tiles of level l (set by the launcher)
@@ -234,5 +237,9 @@ bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_
 bool make_tmap_2d_f32(CUtensorMap* m, const void* ptr, int64_t rows, int D);
 // Dense prefill scoring of one chunk on the tensor cores (grid: tiles, Hsel, batch).
 bool launch_score_tc(const SelectParams& p, dim3 grid, cudaStream_t st);
+// Splits n fp32 values (n % 4 == 0, 16-byte aligned) into a tf32 head (the 13 low mantissa bits
+// cleared) and the exact fp32 remainder, for the two arrays src0 (n0 values) and src1 (n1).
+bool launch_split_tf32(const float* src0, float* hi0, float* lo0, int64_t n0, const float* src1, float* hi1,
+                       float* lo1, int64_t n1, cudaStream_t st);
 
 }  // namespace pisa

@@ -4,21 +4,22 @@
 // fp32 dot products q . node, written to the score plane that descent_kernel
 // reads (same tiling, same plane, same eligibility rule as the FFMA tiles).
 //
-// One CTA per 128 query blocks x 128 nodes. The fp32 operands reach shared
-// memory by 2-D TMA (32 columns x 128 rows per box, 128-byte swizzle), D in
-// chunks of 32 through one stage per CTA; three CTAs share an SM, so one
-// CTA's copies overlap the others' splitting, MMAs and stores. Each value is split there into a tf32
-// head (its top 19 bits) and an exact fp32 remainder, and tcgen05 MMAs of kind
-// tf32 accumulate head*head + head*rest + rest*head in TMEM. The dropped
-// rest*rest term and the remainders' own tf32 rounding are below 2^-21 of
-// |q||node| per product, the size of fp32 rounding over the dot product, so
+// One CTA per 128 query blocks x 128 nodes. Every fp32 operand value x enters
+// as a tf32 head h (x with its 13 low mantissa bits cleared) and the exact fp32
+// remainder r = x - h, written by split_tf32_kernel into the workspace before
+// the tiles run; tcgen05 MMAs of kind tf32 accumulate h*h + h*r + r*h in TMEM.
+// The dropped r*r term and the remainders' own tf32 rounding are below 2^-21
+// of |q||node| per product, the size of fp32 rounding over the dot product, so
 // the ranking the descent draws from these scores differs from an fp32 dot
 // product only where two scores agree to about six digits (a near-tie).
 //
-// Roles: thread 0 issues the copies and the MMAs, all 256 threads split the
-// operands, and the eight warps read the 128 x 128 accumulator out of TMEM
-// (warp w: query blocks 32 (w % 4).., nodes 64 (w / 4)..) and store it through a
-// padded shared tile, 32 consecutive nodes of one row per store instruction.
+// The four operand chunks of 32 columns (heads and remainders of both sides)
+// arrive by 2-D TMA (32 columns x 128 rows per box, 128-byte swizzle) into one
+// 64 KB stage; thread 0 runs the copy-MMA loop over D, and three CTAs share an
+// SM so that one CTA's copies overlap the others' MMAs and stores. The eight
+// warps then read the 128 x 128 accumulator out of TMEM (warp w: query blocks
+// 32 (w % 4).., nodes 64 (w / 4)..) and store it through a padded shared tile,
+// 32 consecutive nodes of one row per store instruction.
 #include <cuda.h>
 
 #include "pisa_device.cuh"
@@ -29,9 +30,8 @@ constexpr int kStTile = 128;                 // query blocks and nodes per tile
 constexpr int kStChunk = 32;                 // D per stage (one 128-byte swizzle atom of fp32)
 constexpr int kStThreads = 256;
 constexpr int kStOp = kStTile * kStChunk * 4;  // one operand chunk: 16 KB
-constexpr int kStStage = 4 * kStOp;            // A head, A rest, B head, B rest
-constexpr int kStStages = 1;                   // one stage: three CTAs share an SM and overlap
-constexpr int kStSmem = 1024 + kStStages * kStStage + 256;
+constexpr int kStStage = 4 * kStOp;            // A head, A remainder, B head, B remainder
+constexpr int kStSmem = 1024 + kStStage + 256;  // three CTAs share an SM
 
 // kind::tf32 instruction descriptor: fp32 accumulator, A and B tf32, both K-major.
 __host__ __device__ constexpr uint32_t idesc_tf32_f32(int m, int n) {
@@ -49,14 +49,14 @@ __device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
-// Splits one loaded operand chunk in place: head = x with its 13 low mantissa bits cleared (exact
-// in tf32), rest = x - head (exact in fp32), written at the same swizzled offsets.
-__device__ __forceinline__ void split_chunk(uint8_t* head, uint8_t* rest, int tid) {
-    float4* h4 = reinterpret_cast<float4*>(head);
-    float4* r4 = reinterpret_cast<float4*>(rest);
-#pragma unroll 4
-    for (int e = tid; e < kStOp / 16; e += kStThreads) {
-        const float4 x = h4[e];
+// head and remainder of n4 float4 values (grid-stride)
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float4* src0, float4* hi0, float4* lo0, int64_t n0,
+                                                         const float4* src1, float4* hi1, float4* lo1, int64_t n1) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n0 + n1; e += stride) {
+        const bool first = e < n0;
+        const int64_t k = first ? e : e - n0;
+        const float4 x = first ? src0[k] : src1[k];
         float4 h, r;
         h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
         h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
@@ -66,9 +66,22 @@ __device__ __forceinline__ void split_chunk(uint8_t* head, uint8_t* rest, int ti
         r.y = x.y - h.y;
         r.z = x.z - h.z;
         r.w = x.w - h.w;
-        h4[e] = h;
-        r4[e] = r;
+        (first ? hi0 : hi1)[k] = h;
+        (first ? lo0 : lo1)[k] = r;
     }
+}
+
+bool launch_split_tf32(const float* src0, float* hi0, float* lo0, int64_t n0, const float* src1, float* hi1,
+                       float* lo1, int64_t n1, cudaStream_t st) {
+    const int64_t n4 = (n0 + n1) / 4;
+    const int64_t want = (n4 + 255) / 256;
+    const int64_t blocks = want < 148 * 8 ? want : 148 * 8;
+    if (blocks <= 0) return true;
+    split_tf32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(src0), reinterpret_cast<float4*>(hi0), reinterpret_cast<float4*>(lo0),
+        n0 / 4, reinterpret_cast<const float4*>(src1), reinterpret_cast<float4*>(hi1), reinterpret_cast<float4*>(lo1),
+        n1 / 4);
+    return cudaGetLastError() == cudaSuccess;
 }
 
 template <int D>
@@ -78,9 +91,9 @@ __global__ void __launch_bounds__(kStThreads, 3)
     constexpr int NC = D / kStChunk;
     extern __shared__ uint8_t st_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(st_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + kStStages * kStStage);  // per stage
-    uint64_t* done = full + kStStages;                                          // per stage: its MMAs completed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + kStStages);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kStStage);  // the stage's copies landed
+    uint64_t* done = full + 1;                                       // the MMAs of the stage completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
     const int hs = blockIdx.y, b = blockIdx.z;
     int tile = blockIdx.x, l = 0;
@@ -102,15 +115,16 @@ __global__ void __launch_bounds__(kStThreads, 3)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kvh = hs / p.gsel_div;
+    // head rows of the tile; the remainder rows follow the whole head array
+    const int qrows = static_cast<int>(gridDim.z) * p.Hsel * p.nqb;
+    const int nrows = static_cast<int>(gridDim.z) * p.Hkv * p.total_nodes;
     const int qrow = static_cast<int>((static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i0);
     const int nrow = static_cast<int>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.total_nodes + p.loff[l] + c0);
     const uint32_t detail_base = kKernSelect << 8;
 
     if (tid == 0) {
-        for (int s = 0; s < kStStages; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(done + s, 1);
-        }
+        mbar_init(full, 1);
+        mbar_init(done, 1);
         fence_barrier_init();
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmN);
@@ -121,35 +135,27 @@ __global__ void __launch_bounds__(kStThreads, 3)
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    auto stage_ptr = [&](int s, int op) { return base + s * kStStage + op * kStOp; };  // op: 0 Ah 1 Ar 2 Bh 3 Br
-    auto load = [&](int c) {
-        const int s = c % kStStages;
-        mbar_arrive_expect_tx(full + s, 2 * kStOp);
-        tma_load_2d(stage_ptr(s, 0), &tmQ, c * kStChunk, qrow, full + s);
-        tma_load_2d(stage_ptr(s, 2), &tmN, c * kStChunk, nrow, full + s);
-    };
-    int loaded = 0;        // thread 0: chunks whose copies were started
-    int last_commit = -1;  // thread 0: last chunk whose MMAs were issued
-    if (tid == 0)
-        for (; loaded < kStStages && loaded < NC; ++loaded) load(loaded);
-
+    auto op_ptr = [&](int op) { return base + op * kStOp; };  // op: 0 A head, 1 A rest, 2 B head, 3 B rest
+    // thread 0 runs the copies and the MMAs: chunk c's copies land, its MMAs run, and once they
+    // have read the stage the next chunk's copies start
     bool ok = true;
-    constexpr uint32_t idesc = idesc_tf32_f32(128, 128);
-    for (int c = 0; c < NC; ++c) {
-        const int s = c % kStStages, use = c / kStStages;
-        if (ok) ok = mbar_wait(full + s, use & 1, p.status, detail_base | 0x41u);
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        split_chunk(stage_ptr(s, 0), stage_ptr(s, 1), tid);
-        split_chunk(stage_ptr(s, 2), stage_ptr(s, 3), tid);
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
+    if (tid == 0) {
+        constexpr uint32_t idesc = idesc_tf32_f32(128, 128);
+        const uint64_t ah = smem_desc_sw128(smem_u32(op_ptr(0)), 16, 1024);
+        const uint64_t ar = smem_desc_sw128(smem_u32(op_ptr(1)), 16, 1024);
+        const uint64_t bh = smem_desc_sw128(smem_u32(op_ptr(2)), 16, 1024);
+        const uint64_t br = smem_desc_sw128(smem_u32(op_ptr(3)), 16, 1024);
+        int loaded = 0, committed = 0;
+        for (int c = 0; c < NC; ++c) {
+            if (c > 0 && !(ok = mbar_wait(done, (c - 1) & 1, p.status, detail_base | 0x42u))) break;
+            mbar_arrive_expect_tx(full, 4 * kStOp);
+            tma_load_2d(op_ptr(0), &tmQ, c * kStChunk, qrow, full);
+            tma_load_2d(op_ptr(1), &tmQ, c * kStChunk, qrow + qrows, full);
+            tma_load_2d(op_ptr(2), &tmN, c * kStChunk, nrow, full);
+            tma_load_2d(op_ptr(3), &tmN, c * kStChunk, nrow + nrows, full);
+            ++loaded;
+            if (!(ok = mbar_wait(full, c & 1, p.status, detail_base | 0x41u))) break;
             tc_fence_after();
-            const uint64_t ah = smem_desc_sw128(smem_u32(stage_ptr(s, 0)), 16, 1024);
-            const uint64_t ar = smem_desc_sw128(smem_u32(stage_ptr(s, 1)), 16, 1024);
-            const uint64_t bh = smem_desc_sw128(smem_u32(stage_ptr(s, 2)), 16, 1024);
-            const uint64_t br = smem_desc_sw128(smem_u32(stage_ptr(s, 3)), 16, 1024);
 #pragma unroll
             for (int ks = 0; ks < kStChunk / 8; ++ks) {
                 const uint32_t off = static_cast<uint32_t>((ks * 32) >> 4);  // 8 tf32 = 32 bytes per K step
@@ -157,28 +163,13 @@ __global__ void __launch_bounds__(kStThreads, 3)
                 mma_tf32_ss(tm, ah + off, br + off, idesc, 1u);
                 mma_tf32_ss(tm, ar + off, bh + off, idesc, 1u);
             }
-            mma_commit(done + s);
-            last_commit = c;
-            if (c + kStStages < NC) {
-                // the stage is refilled once its MMAs have read it
-                if (mbar_wait(done + s, use & 1, p.status, detail_base | 0x42u)) {
-                    load(c + kStStages);
-                    ++loaded;
-                } else {
-                    ok = false;
-                }
-            }
+            mma_commit(done);
+            ++committed;
         }
-    }
-    // every MMA issued has completed, and every copy started has landed, before the epilogue and
-    // before shared and tensor memory are released
-    if (tid == 0) {
-        // the last commit covers every MMA issued before it; the last two copies are the only ones
-        // that can still be in flight (their phases are the latest of their barriers)
-        if (last_commit >= 0)
-            mbar_wait(done + last_commit % kStStages, (last_commit / kStStages) & 1, p.status, detail_base | 0x43u);
-        for (int c = max(0, loaded - kStStages); c < loaded; ++c)
-            mbar_wait(full + c % kStStages, (c / kStStages) & 1, p.status, detail_base | 0x44u);
+        // every MMA issued has completed (the last commit covers all), and every copy started has
+        // landed (only the last can be pending), before the epilogue and before memory is released
+        if (committed > 0) mbar_wait(done, (committed - 1) & 1, p.status, detail_base | 0x43u);
+        if (loaded > committed) mbar_wait(full, (loaded - 1) & 1, p.status, detail_base | 0x44u);
     }
     ok = __syncthreads_and(ok);
     tc_fence_after();
@@ -219,8 +210,10 @@ __global__ void __launch_bounds__(kStThreads, 3)
 bool launch_score_tc(const SelectParams& p, dim3 grid, cudaStream_t st) {
     const int64_t qrows = static_cast<int64_t>(grid.z) * p.Hsel * p.nqb;
     const int64_t nrows = static_cast<int64_t>(grid.z) * p.Hkv * p.total_nodes;
+    if (2 * qrows >= (int64_t(1) << 31) || 2 * nrows >= (int64_t(1) << 31)) return false;
     CUtensorMap tq, tn;
-    if (!make_tmap_2d_f32(&tq, p.qbar, qrows, p.D) || !make_tmap_2d_f32(&tn, p.pyr, nrows, p.D)) return false;
+    if (!make_tmap_2d_f32(&tq, p.qsplit, 2 * qrows, p.D) || !make_tmap_2d_f32(&tn, p.nsplit, 2 * nrows, p.D))
+        return false;
     static bool configured[2] = {false, false};
     const int k = p.D == 64 ? 0 : 1;
     if (!configured[k]) {

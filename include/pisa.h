@@ -127,7 +127,10 @@ PISA_API pisa_status pisa_pyramid_size(const pisa_shape *shape, size_t *bytes);
  * holds an fp32 score plane of B * Hsel * qc * total_nodes values (Hsel =
  * heads_kv, or heads_q with select_per_qhead): the selection scores and
  * descends qc query blocks at a time, qc a multiple of 128 chosen so the plane
- * stays within 192 MiB (128 query blocks if even those need more). Host only. */
+ * stays within 192 MiB (128 query blocks if even those need more), and a copy
+ * of the query summaries and of the pyramid split into tf32 head and remainder
+ * (2 * 4 * D * (B * Hsel * nQB + B * heads_kv * total_nodes) bytes) for the
+ * tensor-core scoring. Host only. */
 PISA_API pisa_status pisa_workspace_size(const pisa_shape *shape, size_t *bytes);
 
 /* Step 1, the key pyramid ("Le pooling comme premiere reduction"): level 0 is
