@@ -68,6 +68,7 @@ static_assert(kSmem < (1 << 18), "descriptor start addresses below 2^18");
 
 }  // namespace
 
+template <int BLK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -85,18 +86,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* mma_final = p_ready + kNst;     // 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
 
-    const int j = static_cast<int>(blockIdx.x), kvh = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
+    // 64 keys per CTA: key block j, or half jh of a 128-key block
+    constexpr int HB = BLK / kTB;
+    const int j = static_cast<int>(blockIdx.x) / HB, jh = static_cast<int>(blockIdx.x) % HB;
+    const int kvh = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int plane = b * p.Hkv + kvh;
     const int32_t* offs = p.counts + static_cast<int64_t>(plane) * (p.n0 + 1);
     const int32_t* ent = p.entries + static_cast<int64_t>(plane) * p.max_entries;
     const int e_lo = offs[j], e_hi = offs[j + 1];
-    const int ntiles = (e_hi - e_lo + 1) / 2;
-    const int64_t kbase = static_cast<int64_t>(plane) * p.N + static_cast<int64_t>(j) * kTB;
+    // a tile is 128 query rows: two entries of 64-row query blocks, or one 128-row query block
+    // (its rows 0-63 as the first half, 64-127 as the second)
+    const int ntiles = HB == 1 ? (e_hi - e_lo + 1) / 2 : e_hi - e_lo;
+    const int64_t kbase = static_cast<int64_t>(plane) * p.N + static_cast<int64_t>(j) * BLK + jh * kTB;
     const uint32_t detail_base = kKernAttnBackward << 8;
     // list entry of half `half` of tile t; a missing second entry repeats the last one (its rows
     // get P = dS = 0, and repeating real rows keeps every operand finite)
     auto entry_of = [&](int t, int half) -> int {
+        if (HB == 2) return e_lo + t;
         const int e = e_lo + 2 * t + half;
         return e < e_hi ? e : e_hi - 1;
     };
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int code = ent[entry_of(t, half)];
                     const int i = code / p.g, head = kvh * p.g + code % p.g;
                     const int32_t qrow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + head) * p.N +
-                                                              static_cast<int64_t>(i) * kTB);
+                                                              static_cast<int64_t>(i) * BLK + (HB == 2 ? half * kTB : 0));
 #pragma unroll
                     for (int s = 0; s < kDS; ++s) {
                         tma_load_2d(sq + s * kSub + half * kTB * 128, &tmQ, s * 64, qrow, qo_full + st);
@@ -219,15 +226,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < ntiles; ++t) {
             const int st = t % kNst;
             const uint32_t ph = (t / kNst) & 1;
-            const int e = e_lo + 2 * t + half;
-            const bool valid = e < e_hi;
+            const bool valid = HB == 2 || e_lo + 2 * t + half < e_hi;
             const int code = ent[entry_of(t, half)];
             const int i = code / p.g, head = kvh * p.g + code % p.g;
-            const int64_t row = (static_cast<int64_t>(b) * p.Hq + head) * p.N + static_cast<int64_t>(i) * kTB + tr;
+            const int qt = (HB == 2 ? half * kTB : 0) + tr;  // query position in its block
+            const int64_t row = (static_cast<int64_t>(b) * p.Hq + head) * p.N + static_cast<int64_t>(i) * BLK + qt;
             const float lse2 = p.lse[row] * 1.4426950408889634f;
             const float dlt = p.delta[row];
-            // keys from mask_from on are masked (causal diagonal block), all of them for a padding row
-            const int mask_from = !valid ? 0 : ((p.causal && i == j) ? tr + 1 : kTB);
+            // keys from mask_from on are masked (causal diagonal block: key jh * 64 + u is visible
+            // from query position qt when jh * 64 + u <= qt), all of them for a padding row
+            const int mask_from = !valid ? 0 : ((p.causal && i == j) ? max(0, min(kTB, qt - jh * kTB + 1)) : kTB);
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full + st, ph, p.status, detail_base | 0x20u));
             tc_fence_after();
             uint32_t pk[16], dk[16];  // P and dS of this thread's 32 keys, bf16 pairs
@@ -334,7 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 
 constexpr int kRD = 128;                       // head dim
-constexpr int kRB = 64;                        // block
 constexpr int kRDS = kRD / 64;
 constexpr uint32_t kRSub = 128 * 128;          // [128 rows x 128 B]
 constexpr uint32_t kRTile = kRDS * kRSub;      // Q, dO, or one 128-key K / V group: 32 KB
@@ -360,10 +367,12 @@ static_assert(kRSmem < (1 << 18), "descriptor start addresses below 2^18");
 
 }  // namespace
 
+template <int BLK>
 __global__ void __launch_bounds__(kRThreads, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const BwdParams p, const int gh, const int chunks) {
+    constexpr int GB = 128 / BLK;  // selected blocks per 128-key group
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* aux = base + kROffAux;
@@ -411,14 +420,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
         fence_barrier_init();
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmdO);
-        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * gh * kRB * kRD * 2));
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * gh * BLK * kRD * 2));
         for (int hh = 0; hh < gh; ++hh) {
             const int32_t qrow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
-                                                      static_cast<int64_t>(i) * kRB);
+                                                      static_cast<int64_t>(i) * BLK);
 #pragma unroll
             for (int s = 0; s < kRDS; ++s) {
-                tma_load_2d(base + kROffQ + s * kRSub + hh * kRB * 128, &tmQ, s * 64, qrow, q_full);
-                tma_load_2d(base + kROffO + s * kRSub + hh * kRB * 128, &tmdO, s * 64, qrow, q_full);
+                tma_load_2d(base + kROffQ + s * kRSub + hh * BLK * 128, &tmQ, s * 64, qrow, q_full);
+                tma_load_2d(base + kROffO + s * kRSub + hh * BLK * 128, &tmdO, s * 64, qrow, q_full);
             }
         }
     }
@@ -448,7 +457,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
     const int nsel = *s_nsel;
-    const int ngroups = (nsel + 1) / 2;
+    const int ngroups = (nsel + GB - 1) / GB;
     const int diag_pos = *s_diag;
 
     int issued_last = -1;
@@ -464,14 +473,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             for (int g = 0; g < ngroups; ++g) {
                 const int st = g % nst, use = g / nst;
                 if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
-                const int nb = min(2, nsel - 2 * g);
-                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * kRB * kRD * 2));
+                const int nb = min(GB, nsel - GB * g);
+                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * BLK * kRD * 2));
                 for (int u = 0; u < nb; ++u) {
                     const int32_t krow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N +
-                                                              static_cast<int64_t>(list[2 * g + u]) * kRB);
+                                                              static_cast<int64_t>(list[GB * g + u]) * BLK);
 #pragma unroll
                     for (int s = 0; s < kRDS; ++s)
-                        tma_load_2d(ring + st * kRTile + s * kRSub + u * kRB * 128, tmap, s * 64, krow, full + st);
+                        tma_load_2d(ring + st * kRTile + s * kRSub + u * BLK * 128, tmap, s * 64, krow, full + st);
                 }
                 issued_last = g;
             }
@@ -485,7 +494,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             const uint64_t dKm = smem_desc_sw128(s0 + kROffK, kRSub, 1024);  // K as the MN-major B of dS.K
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kRD, 0, 1);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
-            auto ncols_of = [&](int g) { return min(2, nsel - 2 * g) * kRB; };
+            auto ncols_of = [&](int g) { return min(GB, nsel - GB * g) * BLK; };
             // dP(g) = dO V_g^T into the dP columns (after the elementwise warps read dP(g-1)) and
             // S(g) = Q K_g^T into S buffer g % 2 (after dQ(g-2) read the dS it held); the two chains
             // alternate so the tensor pipe runs them at its independent-MMA rate
@@ -542,19 +551,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
         // ---------------------------------------------------------------- elementwise warps
         const int q = warp % 4, c4 = warp / 4;  // TMEM lane quadrant; keys 32 c4 .. of each group
         const int r = q * 32 + lane;             // row of the tile
-        const bool valid = r < gh * kRB;
-        const int hh = valid ? r / kRB : 0, t = r % kRB;
-        const int64_t grow = (static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N + static_cast<int64_t>(i) * kRB + t;
+        const bool valid = r < gh * BLK;
+        const int hh = valid ? r / BLK : 0, t = r % BLK;
+        const int64_t grow = (static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N + static_cast<int64_t>(i) * BLK + t;
         const float lse2 = p.lse[grow] * 1.4426950408889634f;
         const float dlt = p.delta[grow];
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const float c2 = p.scale_log2;
         bool ok = true;
         for (int g = 0; g < ngroups; ++g) {
-            const int ncols = min(2, nsel - 2 * g) * kRB;
+            const int ncols = min(GB, nsel - GB * g) * BLK;
             const bool mine = c4 * 32 < ncols;  // this quarter of the group holds keys
             // first column of the diagonal block in this group (128: not here)
-            const int diag_lo = (diag_pos >= 0 && diag_pos / 2 == g) ? (diag_pos % 2) * kRB : 128;
+            const int diag_lo = (diag_pos >= 0 && diag_pos / GB == g) ? (diag_pos % GB) * BLK : 128;
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sdp_full, g & 1, p.status, detail_base | 0x20u));
             tc_fence_after();
             const uint32_t s_col = tm + lane_base + kRColS + 128 * (g % 2) + 32 * c4;
@@ -633,34 +642,44 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
 }
 
-bool bwd_dq_tc_supported(const BwdParams& p) { return p.D == kRD && p.blk == kRB && p.topk <= kRMaxList; }
+bool bwd_dq_tc_supported(const BwdParams& p) {
+    return p.D == kRD && (p.blk == 64 || p.blk == 128) && p.topk <= kRMaxList;
+}
 
-bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
-    if (!bwd_dq_tc_supported(p)) return false;
+template <int BLK>
+static bool launch_dq(const BwdParams& p, int32_t batch, cudaStream_t st) {
     CUtensorMap tq, tdo, tk, tv;
     const int64_t qrows = static_cast<int64_t>(batch) * p.Hq * p.N;
     const int64_t krows = static_cast<int64_t>(batch) * p.Hkv * p.N;
-    if (!make_tmap_2d(&tq, p.Q, qrows, kRD, kRB) || !make_tmap_2d(&tdo, p.dO, qrows, kRD, kRB) ||
-        !make_tmap_2d(&tk, p.K, krows, kRD, kRB) || !make_tmap_2d(&tv, p.V, krows, kRD, kRB))
+    if (!make_tmap_2d(&tq, p.Q, qrows, kRD, BLK) || !make_tmap_2d(&tdo, p.dO, qrows, kRD, BLK) ||
+        !make_tmap_2d(&tk, p.K, krows, kRD, BLK) || !make_tmap_2d(&tv, p.V, krows, kRD, BLK))
         return false;
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(bwd_dq_tc_kernel<BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kRSmem)) != cudaSuccess)
             return false;
         configured = true;
     }
+    // 128 rows: two heads of 64-token blocks (one head, 64 rows, when the group is odd), or one head
+    // of 128-token blocks
     const int gsel = p.per_qhead ? 1 : p.g;
-    const int gh = gsel % 2 == 0 ? 2 : 1;  // two heads fill the 128 rows; else one head (64 rows)
+    const int gh = BLK == 128 ? 1 : (gsel % 2 == 0 ? 2 : 1);
     const int chunks = gsel / gh;
-    bwd_dq_tc_kernel<<<dim3(p.nqb, p.Hsel * chunks, batch), kRThreads, kRSmem, st>>>(tq, tdo, tk, tv, p, gh, chunks);
+    bwd_dq_tc_kernel<BLK><<<dim3(p.nqb, p.Hsel * chunks, batch), kRThreads, kRSmem, st>>>(tq, tdo, tk, tv, p, gh,
+                                                                                          chunks);
     return cudaGetLastError() == cudaSuccess;
 }
 
-bool bwd_dkdv_tc_supported(const BwdParams& p) { return p.D == kTD && p.blk == kTB; }
+bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
+    if (!bwd_dq_tc_supported(p)) return false;
+    return p.blk == 128 ? launch_dq<128>(p, batch, st) : launch_dq<64>(p, batch, st);
+}
 
-bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
-    if (!bwd_dkdv_tc_supported(p)) return false;
+bool bwd_dkdv_tc_supported(const BwdParams& p) { return p.D == kTD && (p.blk == 64 || p.blk == 128); }
+
+template <int BLK>
+static bool launch_dkdv(const BwdParams& p, int32_t batch, cudaStream_t st) {
     CUtensorMap tq, tdo, tk, tv;
     const int64_t qrows = static_cast<int64_t>(batch) * p.Hq * p.N;
     const int64_t krows = static_cast<int64_t>(batch) * p.Hkv * p.N;
@@ -669,13 +688,19 @@ bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
         return false;
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmem)) != cudaSuccess)
             return false;
         configured = true;
     }
-    bwd_dkdv_tc_kernel<<<dim3(p.n0, p.Hkv, batch), kThreads, kSmem, st>>>(tq, tdo, tk, tv, p);
+    // one CTA per 64 keys: a 128-key block is taken as its two halves
+    bwd_dkdv_tc_kernel<BLK><<<dim3(p.n0 * (BLK / kTB), p.Hkv, batch), kThreads, kSmem, st>>>(tq, tdo, tk, tv, p);
     return cudaGetLastError() == cudaSuccess;
+}
+
+bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
+    if (!bwd_dkdv_tc_supported(p)) return false;
+    return p.blk == 128 ? launch_dkdv<128>(p, batch, st) : launch_dkdv<64>(p, batch, st);
 }
 
 }  // namespace pisa

@@ -18,7 +18,10 @@ W = workloads.Workload
 CASES = {
     "gqa4-causal": W("bwd-gqa4-causal", 1, 8, 2, 20 * 64, 20 * 64, 128, 64, 4, 5, 1, "iid", 41),
     "gqa4-d64-noncausal": W("bwd-gqa4-d64", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 4, 0, "iid", 42),
+    # head dim 128 with 128-key blocks: tcgen05 in both passes, the column pass taking each key
+    # block as two 64-key halves
     "mha-b128-causal": W("bwd-mha-b128", 1, 2, 2, 12 * 128, 12 * 128, 128, 128, 8, 4, 1, "clustered", 43),
+    "gqa4-b128-noncausal": W("bwd-gqa4-b128", 2, 8, 2, 10 * 128, 10 * 128, 128, 128, 4, 3, 0, "iid", 47),
     "mha-d64-b64-causal": W("bwd-mha-d64", 1, 3, 3, 17 * 64, 17 * 64, 64, 64, 4, 6, 1, "clustered", 44),
     # head dim 128 with 64-key blocks: the column pass runs on the tensor-core (tcgen05) kernel
     "gqa8-d128-noncausal": W("bwd-gqa8-d128", 2, 16, 2, 16 * 64, 16 * 64, 128, 64, 4, 6, 0, "clustered", 45),
@@ -63,17 +66,18 @@ def test_backward_matches_oracle(name, cuda_device):
     _close(dv, ref["dV"], f"{name} dV")
 
 
-def test_backward_per_qhead_and_forced(cuda_device):
-    w = CASES["gqa4-causal"]
+@pytest.mark.parametrize("name", ["gqa4-causal", "gqa4-b128-noncausal"])
+def test_backward_per_qhead_and_forced(name, cuda_device):
+    w = CASES[name]
     shape, (q, k, v, o, lse, do, idx), (dq, dk, dv) = _grads(w, cuda_device, per_qhead=True, forced=3)
     Q, K, V, dO = (gu.host_f32(x) for x in (q, k, v, do))
-    ref = oracle.backward(Q, K, V, dO, idx.cpu().numpy(), w.block, True, per_qhead=True)
+    ref = oracle.backward(Q, K, V, dO, idx.cpu().numpy(), w.block, bool(w.causal), per_qhead=True)
     _close(dq, ref["dQ"], "per-qhead dQ")
     _close(dk, ref["dK"], "per-qhead dK")
     _close(dv, ref["dV"], "per-qhead dV")
 
 
-@pytest.mark.parametrize("name", ["mha-d64-b64-causal", "mha-d128-b64-causal"])
+@pytest.mark.parametrize("name", ["mha-d64-b64-causal", "mha-d128-b64-causal", "mha-b128-causal"])
 def test_backward_full_topk_is_dense_gradient(name, cuda_device):
     """K = every block: the gradient of dense causal softmax attention (every key block's
     inverse list then holds every later query block)."""
