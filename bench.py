@@ -568,7 +568,7 @@ def run_backward(args, world, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": "sparse-attn backward tokens/s at N=128K (dQ, dK, dV through the forward's selection)",
+        "metric": f"sparse-attn backward tokens/s on {w.name} (dQ, dK, dV through the forward's selection)",
         "value": whole_job_tokens_per_s(w.batch * w.seq_q, world, ms_step),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",

@@ -1,10 +1,13 @@
-// Backward column pass on the tensor cores (sm_100a): dK and dV of one 64-key
-// block through a fixed selection (PISA page, section "Ce que cela change pour
-// vous": the sparse kernels serve training; the selection has no gradient).
+// Backward on the tensor cores (sm_100a), both passes, through a fixed selection
+// (PISA page, section "Ce que cela change pour vous": the sparse kernels serve
+// training; the selection has no gradient). Head dim 64 or 128; 64- or 128-key
+// blocks.
 //
-// One CTA per (batch, KV head, key block j). Its inverse list (the query blocks
-// and query heads whose selection holds j, ascending) is taken two entries at a
-// time: a tile of 128 query rows. Per tile, with the forward's LSE and
+// Column pass: dK and dV of 64 keys. One CTA per (batch, KV head, key block j)
+// for 64-key blocks, per (batch, KV head, half of key block j) for 128-key
+// blocks. Its inverse list (the query blocks and query heads whose selection
+// holds j, ascending) makes tiles of 128 query rows: two entries of 64-row query
+// blocks, or one 128-row query block. Per tile, with the forward's LSE and
 // Delta = rowsum(dO * O):
 //   S  = Q K_j^T,  dP = dO V_j^T            tcgen05, M = 128 rows, N = 64 keys, fp32 in TMEM
 //                                           (separate barriers: P is computed while dP forms)
@@ -34,8 +37,8 @@ namespace pisa {
 
 namespace {
 
-constexpr int kTD = 128;                        // head dim
-constexpr int kTB = 64;                         // keys per block
+constexpr int kTD = 128;                        // largest head dim (the shared-memory layout's)
+constexpr int kTB = 64;                         // keys per CTA
 constexpr int kDS = kTD / 64;                   // 128-byte column tiles along the head dim
 constexpr uint32_t kSub = 128 * 128;            // [128 rows x 128 B] tile
 constexpr uint32_t kKSub = kTB * 128;           // [64 keys x 128 B] tile
@@ -68,7 +71,7 @@ static_assert(kSmem < (1 << 18), "descriptor start addresses below 2^18");
 
 }  // namespace
 
-template <int BLK>
+template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -88,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // 64 keys per CTA: key block j, or half jh of a 128-key block
     constexpr int HB = BLK / kTB;
+    constexpr int DS = D / 64;  // 128-byte column tiles loaded per row
     const int j = static_cast<int>(blockIdx.x) / HB, jh = static_cast<int>(blockIdx.x) % HB;
     const int kvh = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,16 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && ntiles > 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmdO);
-            mbar_arrive_expect_tx(kv_full, 2 * kKVBytes);
+            mbar_arrive_expect_tx(kv_full, 2 * DS * kKSub);
 #pragma unroll
-            for (int s = 0; s < kDS; ++s) {
+            for (int s = 0; s < DS; ++s) {
                 tma_load_2d(base + kOffK + s * kKSub, &tmK, s * 64, static_cast<int32_t>(kbase), kv_full);
                 tma_load_2d(base + kOffV + s * kKSub, &tmV, s * 64, static_cast<int32_t>(kbase), kv_full);
             }
             for (int t = 0; t < ntiles; ++t) {
                 const int st = t % kNst, use = t / kNst;
                 if (!mbar_wait(qo_empty + st, (use & 1) ^ 1, p.status, detail_base | 0x01u)) break;
-                mbar_arrive_expect_tx(qo_full + st, 2 * kQOBytes);
+                mbar_arrive_expect_tx(qo_full + st, 2 * 2 * DS * kTB * 128);
                 uint8_t* sq = base + kOffQ + st * 2 * kQOBytes;
                 for (int half = 0; half < 2; ++half) {
                     const int code = ent[entry_of(t, half)];
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t qrow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + head) * p.N +
                                                               static_cast<int64_t>(i) * BLK + (HB == 2 ? half * kTB : 0));
 #pragma unroll
-                    for (int s = 0; s < kDS; ++s) {
+                    for (int s = 0; s < DS; ++s) {
                         tma_load_2d(sq + s * kSub + half * kTB * 128, &tmQ, s * 64, qrow, qo_full + st);
                         tma_load_2d(sq + kQOBytes + s * kSub + half * kTB * 128, &tmdO, s * 64, qrow, qo_full + st);
                     }
@@ -178,20 +182,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint64_t dq = dmove(dQk, st * 2 * kQOBytes), dout = dmove(dq, kQOBytes);
 #pragma unroll
-                    for (int ks = 0; ks < kTD / 16; ++ks) {
+                    for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t oa = (ks / 4) * kSub + (ks % 4) * 32, ob = (ks / 4) * kKSub + (ks % 4) * 32;
                         mma_bf16_ss(tm + kColS + 64 * st, dmove(dq, oa), dmove(dK, ob), idesc_s, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(s_full + st);  // the exponentials start while dP is formed
 #pragma unroll
-                    for (int ks = 0; ks < kTD / 16; ++ks) {
+                    for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t oa = (ks / 4) * kSub + (ks % 4) * 32, ob = (ks / 4) * kKSub + (ks % 4) * 32;
                         mma_bf16_ss(tm + kColDP + 64 * st, dmove(dout, oa), dmove(dV, ob), idesc_s, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(dp_full + st);
                 }
                 // dV^T += dO^T P and dK^T += Q^T dS: the head dim is M (two 64-column tiles LBO
-                // apart), the 128 rows are K (16 per MMA), the keys N
+                // apart), the 128 rows are K (16 per MMA), the keys N. At head dim 64 the second
+                // tile is never loaded: M stays 128 (an M = 64 MMA takes as long), TMEM lanes
+                // 64-127 receive products of whatever that shared memory holds, and are not read
                 for (int u = r0; ok && u < r1; ++u) {
                     const int su = u % kNst;
                     if (!(ok = mbar_wait(p_ready + su, (u / kNst) & 1, p.status, detail_base | 0x13u))) break;
@@ -283,11 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && ntiles > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(mma_final, 0, p.status, detail_base | 0x22u));
         tc_fence_after();
         const int d = r;
-        __nv_bfloat16* dv_col = p.dV + kbase * kTD + d;
-        __nv_bfloat16* dk_col = p.dK + kbase * kTD + d;
+        __nv_bfloat16* dv_col = p.dV + kbase * D + d;
+        __nv_bfloat16* dk_col = p.dK + kbase * D + d;
         const float sc = p.scale;
         uint32_t v[32], k[32];
-        if (ntiles > 0) {
+        if (ntiles > 0 && (warp % 4) * 32 < D) {
             tmem_ld32(tm + lane_base + kColDV + 32 * ch, v);
             tmem_ld32(tm + lane_base + kColDK + 32 * ch, k);
             tmem_wait_ld();
@@ -295,12 +301,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int x = 0; x < 32; ++x) v[x] = k[x] = 0u;
         }
-        if (ok) {
+        if (ok && d < D) {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
                 const int64_t key = 32 * ch + x;
-                dv_col[key * kTD] = __float2bfloat16_rn(__uint_as_float(v[x]));
-                dk_col[key * kTD] = __float2bfloat16_rn(__uint_as_float(k[x]) * sc);
+                dv_col[key * D] = __float2bfloat16_rn(__uint_as_float(v[x]));
+                dk_col[key * D] = __float2bfloat16_rn(__uint_as_float(k[x]) * sc);
             }
         }
     }
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // issue and TMEM allocation.
 namespace {
 
-constexpr int kRD = 128;                       // head dim
+constexpr int kRD = 128;                       // largest head dim (the shared-memory layout's)
 constexpr int kRDS = kRD / 64;
 constexpr uint32_t kRSub = 128 * 128;          // [128 rows x 128 B]
 constexpr uint32_t kRTile = kRDS * kRSub;      // Q, dO, or one 128-key K / V group: 32 KB
@@ -367,12 +373,13 @@ static_assert(kRSmem < (1 << 18), "descriptor start addresses below 2^18");
 
 }  // namespace
 
-template <int BLK>
+template <int D, int BLK>
 __global__ void __launch_bounds__(kRThreads, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const BwdParams p, const int gh, const int chunks) {
     constexpr int GB = 128 / BLK;  // selected blocks per 128-key group
+    constexpr int DS = D / 64;     // 128-byte column tiles loaded per row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* aux = base + kROffAux;
@@ -420,12 +427,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
         fence_barrier_init();
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmdO);
-        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * gh * BLK * kRD * 2));
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * gh * BLK * D * 2));
         for (int hh = 0; hh < gh; ++hh) {
             const int32_t qrow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + head0 + hh) * p.N +
                                                       static_cast<int64_t>(i) * BLK);
 #pragma unroll
-            for (int s = 0; s < kRDS; ++s) {
+            for (int s = 0; s < DS; ++s) {
                 tma_load_2d(base + kROffQ + s * kRSub + hh * BLK * 128, &tmQ, s * 64, qrow, q_full);
                 tma_load_2d(base + kROffO + s * kRSub + hh * BLK * 128, &tmdO, s * 64, qrow, q_full);
             }
@@ -474,12 +481,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 const int st = g % nst, use = g / nst;
                 if (!mbar_wait(empty + st, (use & 1) ^ 1, p.status, detail_base | (is_k ? 0x01u : 0x02u))) break;
                 const int nb = min(GB, nsel - GB * g);
-                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * BLK * kRD * 2));
+                mbar_arrive_expect_tx(full + st, static_cast<uint32_t>(nb * BLK * D * 2));
                 for (int u = 0; u < nb; ++u) {
                     const int32_t krow = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N +
                                                               static_cast<int64_t>(list[GB * g + u]) * BLK);
 #pragma unroll
-                    for (int s = 0; s < kRDS; ++s)
+                    for (int s = 0; s < DS; ++s)
                         tma_load_2d(ring + st * kRTile + s * kRSub + u * BLK * 128, tmap, s * 64, krow, full + st);
                 }
                 issued_last = g;
@@ -492,7 +499,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             const uint64_t dQk = smem_desc_sw128(s0 + kROffQ, 16, 1024), dOk = smem_desc_sw128(s0 + kROffO, 16, 1024);
             const uint64_t dKk = smem_desc_sw128(s0 + kROffK, 16, 1024), dVk = smem_desc_sw128(s0 + kROffV, 16, 1024);
             const uint64_t dKm = smem_desc_sw128(s0 + kROffK, kRSub, 1024);  // K as the MN-major B of dS.K
-            constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kRD, 0, 1);
+            constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
             bool ok = mbar_wait(q_full, 0, p.status, detail_base | 0x10u);
             auto ncols_of = [&](int g) { return min(GB, nsel - GB * g) * BLK; };
             // dP(g) = dO V_g^T into the dP columns (after the elementwise warps read dP(g-1)) and
@@ -509,7 +516,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 const uint64_t dv = dmove(dVk, sv * kRTile), dk = dmove(dKk, sk * kRTile);
                 const uint32_t s_col = tm + kRColS + 128 * (g % 2);
 #pragma unroll
-                for (int ks = 0; ks < kRD / 16; ++ks) {
+                for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (ks / 4) * kRSub + (ks % 4) * 32;
                     mma_bf16_ss(tm + kRColDP, dmove(dOk, off), dmove(dv, off), id, ks > 0 ? 1u : 0u);
                     mma_bf16_ss(s_col, dmove(dQk, off), dmove(dk, off), id, ks > 0 ? 1u : 0u);
@@ -598,9 +605,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
         for (int g = max(0, ngroups - 2); ok && g < ngroups; ++g)
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(dq_done, g & 1, p.status, detail_base | 0x22u));
         tc_fence_after();
-        if (ok && valid) {
+        if (ok && valid && c4 * 32 < D) {
             const float sc = p.scale;
-            uint4* dst = reinterpret_cast<uint4*>(p.dQ + grow * kRD + c4 * 32);
+            uint4* dst = reinterpret_cast<uint4*>(p.dQ + grow * D + c4 * 32);
             uint32_t o[32];
             if (ngroups > 0) {
                 tmem_ld32(tm + lane_base + kRColDQ + c4 * 32, o);
@@ -643,20 +650,20 @@ __global__ void __launch_bounds__(kRThreads, 1)
 }
 
 bool bwd_dq_tc_supported(const BwdParams& p) {
-    return p.D == kRD && (p.blk == 64 || p.blk == 128) && p.topk <= kRMaxList;
+    return (p.D == 64 || p.D == 128) && (p.blk == 64 || p.blk == 128) && p.topk <= kRMaxList;
 }
 
-template <int BLK>
+template <int D, int BLK>
 static bool launch_dq(const BwdParams& p, int32_t batch, cudaStream_t st) {
     CUtensorMap tq, tdo, tk, tv;
     const int64_t qrows = static_cast<int64_t>(batch) * p.Hq * p.N;
     const int64_t krows = static_cast<int64_t>(batch) * p.Hkv * p.N;
-    if (!make_tmap_2d(&tq, p.Q, qrows, kRD, BLK) || !make_tmap_2d(&tdo, p.dO, qrows, kRD, BLK) ||
-        !make_tmap_2d(&tk, p.K, krows, kRD, BLK) || !make_tmap_2d(&tv, p.V, krows, kRD, BLK))
+    if (!make_tmap_2d(&tq, p.Q, qrows, D, BLK) || !make_tmap_2d(&tdo, p.dO, qrows, D, BLK) ||
+        !make_tmap_2d(&tk, p.K, krows, D, BLK) || !make_tmap_2d(&tv, p.V, krows, D, BLK))
         return false;
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dq_tc_kernel<BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(bwd_dq_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kRSmem)) != cudaSuccess)
             return false;
         configured = true;
@@ -666,41 +673,43 @@ static bool launch_dq(const BwdParams& p, int32_t batch, cudaStream_t st) {
     const int gsel = p.per_qhead ? 1 : p.g;
     const int gh = BLK == 128 ? 1 : (gsel % 2 == 0 ? 2 : 1);
     const int chunks = gsel / gh;
-    bwd_dq_tc_kernel<BLK><<<dim3(p.nqb, p.Hsel * chunks, batch), kRThreads, kRSmem, st>>>(tq, tdo, tk, tv, p, gh,
-                                                                                          chunks);
+    bwd_dq_tc_kernel<D, BLK><<<dim3(p.nqb, p.Hsel * chunks, batch), kRThreads, kRSmem, st>>>(tq, tdo, tk, tv, p,
+                                                                                             gh, chunks);
     return cudaGetLastError() == cudaSuccess;
 }
 
 bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
     if (!bwd_dq_tc_supported(p)) return false;
-    return p.blk == 128 ? launch_dq<128>(p, batch, st) : launch_dq<64>(p, batch, st);
+    if (p.D == 128) return p.blk == 128 ? launch_dq<128, 128>(p, batch, st) : launch_dq<128, 64>(p, batch, st);
+    return p.blk == 128 ? launch_dq<64, 128>(p, batch, st) : launch_dq<64, 64>(p, batch, st);
 }
 
-bool bwd_dkdv_tc_supported(const BwdParams& p) { return p.D == kTD && (p.blk == 64 || p.blk == 128); }
+bool bwd_dkdv_tc_supported(const BwdParams& p) { return (p.D == 64 || p.D == 128) && (p.blk == 64 || p.blk == 128); }
 
-template <int BLK>
+template <int D, int BLK>
 static bool launch_dkdv(const BwdParams& p, int32_t batch, cudaStream_t st) {
     CUtensorMap tq, tdo, tk, tv;
     const int64_t qrows = static_cast<int64_t>(batch) * p.Hq * p.N;
     const int64_t krows = static_cast<int64_t>(batch) * p.Hkv * p.N;
-    if (!make_tmap_2d(&tq, p.Q, qrows, kTD, kTB) || !make_tmap_2d(&tdo, p.dO, qrows, kTD, kTB) ||
-        !make_tmap_2d(&tk, p.K, krows, kTD, kTB) || !make_tmap_2d(&tv, p.V, krows, kTD, kTB))
+    if (!make_tmap_2d(&tq, p.Q, qrows, D, kTB) || !make_tmap_2d(&tdo, p.dO, qrows, D, kTB) ||
+        !make_tmap_2d(&tk, p.K, krows, D, kTB) || !make_tmap_2d(&tv, p.V, krows, D, kTB))
         return false;
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmem)) != cudaSuccess)
             return false;
         configured = true;
     }
     // one CTA per 64 keys: a 128-key block is taken as its two halves
-    bwd_dkdv_tc_kernel<BLK><<<dim3(p.n0 * (BLK / kTB), p.Hkv, batch), kThreads, kSmem, st>>>(tq, tdo, tk, tv, p);
+    bwd_dkdv_tc_kernel<D, BLK><<<dim3(p.n0 * (BLK / kTB), p.Hkv, batch), kThreads, kSmem, st>>>(tq, tdo, tk, tv, p);
     return cudaGetLastError() == cudaSuccess;
 }
 
 bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st) {
     if (!bwd_dkdv_tc_supported(p)) return false;
-    return p.blk == 128 ? launch_dkdv<128>(p, batch, st) : launch_dkdv<64>(p, batch, st);
+    if (p.D == 128) return p.blk == 128 ? launch_dkdv<128, 128>(p, batch, st) : launch_dkdv<128, 64>(p, batch, st);
+    return p.blk == 128 ? launch_dkdv<64, 128>(p, batch, st) : launch_dkdv<64, 64>(p, batch, st);
 }
 
 }  // namespace pisa

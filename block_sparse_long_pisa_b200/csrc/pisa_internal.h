@@ -224,11 +224,11 @@ bool launch_attn_prefill_dual(int D, int blk, const CUtensorMap& q, const CUtens
                               const AttnParams& p, dim3 grid, cudaStream_t st);
 bool launch_attn_decode(const Plan& pl, const DecodeParams& p, cudaStream_t st, int32_t* launches);
 bool launch_attn_backward(const BwdParams& p, int32_t batch, cudaStream_t st, int32_t* launches);
-// Backward column pass on the tensor cores (head dim 128, 64-key blocks); false when the shape is
-// another one or on a launch error.
+// Backward column pass (dK, dV) on the tensor cores (head dim 64 or 128, 64- or 128-key blocks:
+// every shape the library accepts); false when the shape is another one or on a launch error.
 bool bwd_dkdv_tc_supported(const BwdParams& p);
 bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
-// Backward row pass (dQ) on the tensor cores, same shapes.
+// Backward row pass (dQ) on the tensor cores, same shapes (and K up to the prefill limit).
 bool bwd_dq_tc_supported(const BwdParams& p);
 bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.

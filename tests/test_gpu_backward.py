@@ -18,12 +18,12 @@ W = workloads.Workload
 CASES = {
     "gqa4-causal": W("bwd-gqa4-causal", 1, 8, 2, 20 * 64, 20 * 64, 128, 64, 4, 5, 1, "iid", 41),
     "gqa4-d64-noncausal": W("bwd-gqa4-d64", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 4, 0, "iid", 42),
-    # head dim 128 with 128-key blocks: tcgen05 in both passes, the column pass taking each key
-    # block as two 64-key halves
+    # every shape runs both passes on tcgen05; the column pass takes a 128-key block as two
+    # 64-key halves, and at head dim 64 pads the head-dim side of its MMAs to 128 lanes
     "mha-b128-causal": W("bwd-mha-b128", 1, 2, 2, 12 * 128, 12 * 128, 128, 128, 8, 4, 1, "clustered", 43),
     "gqa4-b128-noncausal": W("bwd-gqa4-b128", 2, 8, 2, 10 * 128, 10 * 128, 128, 128, 4, 3, 0, "iid", 47),
     "mha-d64-b64-causal": W("bwd-mha-d64", 1, 3, 3, 17 * 64, 17 * 64, 64, 64, 4, 6, 1, "clustered", 44),
-    # head dim 128 with 64-key blocks: the column pass runs on the tensor-core (tcgen05) kernel
+    "gqa2-d64-b128-causal": W("bwd-gqa2-d64-b128", 1, 4, 2, 10 * 128, 10 * 128, 64, 128, 4, 3, 1, "clustered", 48),
     "gqa8-d128-noncausal": W("bwd-gqa8-d128", 2, 16, 2, 16 * 64, 16 * 64, 128, 64, 4, 6, 0, "clustered", 45),
     "mha-d128-b64-causal": W("bwd-mha-d128", 1, 2, 2, 15 * 64, 15 * 64, 128, 64, 4, 4, 1, "iid", 46),
 }
@@ -66,7 +66,7 @@ def test_backward_matches_oracle(name, cuda_device):
     _close(dv, ref["dV"], f"{name} dV")
 
 
-@pytest.mark.parametrize("name", ["gqa4-causal", "gqa4-b128-noncausal"])
+@pytest.mark.parametrize("name", ["gqa4-causal", "gqa4-b128-noncausal", "gqa4-d64-noncausal"])
 def test_backward_per_qhead_and_forced(name, cuda_device):
     w = CASES[name]
     shape, (q, k, v, o, lse, do, idx), (dq, dk, dv) = _grads(w, cuda_device, per_qhead=True, forced=3)
