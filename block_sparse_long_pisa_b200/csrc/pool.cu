@@ -212,9 +212,12 @@ __global__ void __launch_bounds__(512) pyramid_subtree_kernel(const SubtreeParam
     }
 }
 
-// Levels m+1 .. L-1 of one plane per CTA, level after level, from the rows below in global memory
-// (the subtree roots, then this CTA's own output).
-__global__ void __launch_bounds__(512) pyramid_top_kernel(const SubtreeParams p) {
+// Levels m+1 .. L-1 of one plane per CTA, level after level. With `in_smem`, the subtree roots
+// (level m) are read into shared memory once and every level above is formed there (and written
+// out), so the chain after the subtree grid is one round of global loads; otherwise each level
+// reads the one below from global memory (planes whose top levels exceed the shared memory).
+__global__ void __launch_bounds__(512) pyramid_top_kernel(const SubtreeParams p, const bool in_smem) {
+    extern __shared__ __align__(16) float top[];  // [rows of levels m .. L-1][D] when in_smem
     // launched as a programmatic dependent of the subtree kernel: wait until that grid has
     // completed and its writes are visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -223,14 +226,24 @@ __global__ void __launch_bounds__(512) pyramid_top_kernel(const SubtreeParams p)
     int64_t width_below = 1;
     for (int l = 1; l <= p.m; ++l) width_below *= p.factor;
     const int q4 = p.D / 4;
+    const float* below = out_plane + static_cast<int64_t>(p.loff[p.m]) * p.D;
+    if (in_smem) {
+        const float4* src = reinterpret_cast<const float4*>(below);
+        for (int e = threadIdx.x; e < p.lsize[p.m] * q4; e += blockDim.x) reinterpret_cast<float4*>(top)[e] = src[e];
+        __syncthreads();
+        below = top;
+    }
     for (int l = p.m + 1; l < p.L; ++l) {
-        const float* below = out_plane + static_cast<int64_t>(p.loff[l - 1]) * p.D;
+        float* cur = in_smem ? const_cast<float*>(below) + static_cast<int64_t>(p.lsize[l - 1]) * p.D : nullptr;
+        float* dst = out_plane + static_cast<int64_t>(p.loff[l]) * p.D;
         for (int e = threadIdx.x; e < p.lsize[l] * q4; e += blockDim.x) {
             const int c = e / q4, q = e % q4;
             const float4 v = node_mean4(below + 4 * q, 0, p.D, c, p.factor, p.lsize[l - 1], width_below, p.n0);
-            *reinterpret_cast<float4*>(out_plane + (static_cast<int64_t>(p.loff[l]) + c) * p.D + 4 * q) = v;
+            *reinterpret_cast<float4*>(dst + static_cast<int64_t>(c) * p.D + 4 * q) = v;
+            if (in_smem) *reinterpret_cast<float4*>(cur + static_cast<int64_t>(c) * p.D + 4 * q) = v;
         }
         width_below *= p.factor;
+        below = in_smem ? cur : dst;
         __syncthreads();
     }
 }
@@ -245,6 +258,10 @@ bool launch_block_mean(const MeanParams& p, cudaStream_t st) {
         block_mean_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess;
 }
+
+// Shared memory the top-level kernel may take for a plane's levels m .. L-1 (beyond it, each level
+// reads the one below from global memory).
+constexpr size_t kTopSmemLimit = 160 * 1024;
 
 bool launch_pyramid_two_pass(const SubtreeParams& p, cudaStream_t st, int32_t* launches) {
     const int warps = p.S < 16 ? p.S : 16;
@@ -269,16 +286,25 @@ bool launch_pyramid_two_pass(const SubtreeParams& p, cudaStream_t st, int32_t* l
     ++*launches;
     if (cudaGetLastError() != cudaSuccess) return false;
     if (p.m + 1 < p.L) {
+        size_t top_rows = 0;
+        for (int l = p.m; l < p.L; ++l) top_rows += static_cast<size_t>(p.lsize[l]);
+        const size_t top_smem = top_rows * p.D * sizeof(float);
+        const bool in_smem = top_smem <= kTopSmemLimit;
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(static_cast<unsigned>(p.planes));
         cfg.blockDim = dim3(512);
+        cfg.dynamicSmemBytes = in_smem ? top_smem : 0;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, pyramid_top_kernel, p) != cudaSuccess) return false;
+        if (in_smem && top_smem > 48 * 1024 &&
+            cudaFuncSetAttribute(pyramid_top_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kTopSmemLimit)) != cudaSuccess)
+            return false;
+        if (cudaLaunchKernelEx(&cfg, pyramid_top_kernel, p, in_smem) != cudaSuccess) return false;
         ++*launches;
     }
     return cudaGetLastError() == cudaSuccess;

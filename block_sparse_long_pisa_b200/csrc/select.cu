@@ -1,19 +1,25 @@
 // Pyramid-guided top-K selection ("La selection top-K guidee par la pyramide",
 // PISA page). One CTA of 128 threads per (batch, selection row, query block).
 //
-// 1. The query summary (fp32, computed by the pooling kernel) goes to shared
-//    memory.
+// 1. Each lane holds its slice of the query summary (fp32, computed by the
+//    pooling kernel), loaded from global memory alongside the first nodes.
 // 2. Causal: the node that straddles the query block at each level is
 //    summarised by the mean of its eligible level-0 blocks, built bottom-up
 //    from the pyramid (full children left of the straddling child, plus the
 //    straddling child's own partial sum), so no future key enters a score.
+//    When no level has such a node (decode over a whole cache whose length is
+//    a multiple of every level's width, for one) the step is skipped.
 // 3. The descent starts at the coarsest level whose eligible nodes outnumber
 //    that level's budget: every level above it keeps all its nodes, so its
 //    children are exactly the eligible nodes of this level, and skipping the
 //    coarser scores changes nothing.
 // 4. At each level every candidate gets an fp32 dot product with the query
 //    summary (eight lanes per candidate, so each warp load covers four whole
-//    128-byte lines of node vectors; a three-step shuffle adds the lanes). Candidates are ranked by
+//    128-byte lines of node vectors; a three-step shuffle adds the lanes). The
+//    16 groups of eight lanes issue the loads of four candidates each before
+//    any arithmetic. (Measured at 64 sequences x 8 KV heads over 128K keys:
+//    CTAs of 256 or 512 threads, which score a level in fewer rounds, take
+//    1.3x and 2x as long, since fewer of them are resident per SM.) Candidates are ranked by
 //    a 64-bit key (order-preserving score bits, then inverted node index): higher score first
 //    and, on equal scores, lower index. One warp finds the K_l-th largest key by bisection with
 //    warp-wide counts (the score word first, the index word only when scores tie at the cut;
@@ -65,8 +71,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                         // [cap]
     int32_t* cand = reinterpret_cast<int32_t*>(keys + cap);                    // [cap]
     int32_t* kept = cand + cap;                                                // [cap]
-    float* qs = reinterpret_cast<float*>(kept + cap);                          // [D]
-    float* part = qs + D;                                                      // [L][D]
+    float* part = reinterpret_cast<float*>(kept + cap);                        // [L][D]
     __shared__ int s_nvalid;
     __shared__ float s_margin;
     __shared__ int s_scan[1];   // kept count of the level
@@ -78,9 +83,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     const float* plane = p.pyr + (static_cast<int64_t>(b) * p.Hkv + kvh) * p.total_nodes * D;
     const int64_t row = (static_cast<int64_t>(b) * p.Hsel + hs) * p.nqb + i;
 
-    for (int d = tid; d < D; d += kSelThreads) qs[d] = p.qbar[row * D + d];
-    // partial (straddling) node summaries, bottom-up
-    for (int d = tid; d < D; d += kSelThreads) {
+    // this lane's slice of the query summary: dims 32k + 4*sub .. +3 (its loads overlap the rest
+    // of the set-up and the first level's node loads)
+    const int sub = tid & 7;
+    float4 qv[D / 32];
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) qv[k] = *reinterpret_cast<const float4*>(p.qbar + row * D + 32 * k + 4 * sub);
+    // partial (straddling) node summaries, bottom-up, where some level has a partial node
+    bool any_part = false;
+    for (int l = 1; l < p.L; ++l) {
+        const int64_t c_part = div_width(p, last, l);
+        any_part |= min((c_part + 1) * p.width[l], static_cast<int64_t>(p.n0)) - 1 > last;
+    }
+    for (int d = tid; any_part && d < D; d += kSelThreads) {
         float sum = plane[static_cast<int64_t>(p.loff[0] + last) * D + d];
         for (int l = 1; l < p.L; ++l) {
             const int64_t wl = p.width[l], wb = p.width[l - 1];
@@ -101,11 +116,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     }
     if (tid == 0) s_margin = __int_as_float(0x7F800000);  // +inf
     __syncthreads();
-    // this lane's slice of the query summary: dims 32k + 4*sub .. +3
-    const int sub = tid & 7;
-    float4 qv[D / 32];
-#pragma unroll
-    for (int k = 0; k < D / 32; ++k) qv[k] = *reinterpret_cast<const float4*>(qs + 32 * k + 4 * sub);
 
     // coarsest level whose eligible nodes exceed its budget
     int l0 = -1;
@@ -293,11 +303,11 @@ bool launch_select(const SelectParams& p, int32_t batch, cudaStream_t st, int32_
     for (int l = 0; l < p.L; ++l) maxb = max(maxb, p.budget[l]);
     int cap = 1;
     while (cap < max(p.factor * maxb, p.lsize[p.L - 1])) cap <<= 1;
-    if (cap < 4) cap = 4;  // keeps the fp32 query row 16-byte aligned
+    if (cap < 4) cap = 4;  // keeps the fp32 partial-node rows 16-byte aligned
     if (p.scores != nullptr && !p.decode && dense_select_cap(cap) > 0) return launch_select_dense(p, batch, cap, st, launches);
     *launches += 1;
     const size_t smem = static_cast<size_t>(cap) * (sizeof(uint64_t) + 2 * sizeof(int32_t)) +
-                        static_cast<size_t>(p.D) * (1 + p.L) * sizeof(float);
+                        static_cast<size_t>(p.D) * p.L * sizeof(float);
     dim3 grid(p.nqb, p.Hsel, batch);
     if (p.D == 64) {
         cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
