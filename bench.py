@@ -58,6 +58,19 @@ def kernel_source_hash(sources) -> str:
 ATTN_SOURCES = ("block_sparse_long_pisa_b200/csrc/attn_prefill.cu", "block_sparse_long_pisa_b200/csrc/pisa_device.cuh")
 
 
+def attention_kernel_name(shape) -> str:
+    """The prefill attention kernel the library launches for this shape: a CTA takes the largest
+    divisor of the group whose rows fit two 128-row tiles (one for 128-key blocks; one head under
+    per-query-head selection); units of at most 128 rows run two per CTA."""
+    g = 1 if shape.select_per_qhead else shape.heads_q // shape.heads_kv
+    max_rows = 128 if shape.block == 128 else 256
+    gh = max(d for d in range(1, g + 1) if g % d == 0 and d * shape.block <= max_rows)
+    nm = 2 if gh * shape.block > 128 else 1
+    if nm == 1 and shape.n_qblocks >= 2:
+        return f"attn_prefill_dual_kernel<{shape.head_dim},{shape.block}>"
+    return f"attn_prefill_kernel<{shape.head_dim},{shape.block},{nm}>"
+
+
 def profiled_traffic(kernel_file: str, sources) -> float | None:
     """dram bytes per full-size launch recorded from an ncu capture (profiles/<file>, JSON), or None
     when absent or when the kernel sources have changed since the capture (sha256 prefix recorded
@@ -394,8 +407,9 @@ def run_gpu(args, world, rank, local):
     near_ties = {"rows": int(marg.numel()), "gpu_margin_below_1e-3": near_gpu}
     if cpu is not None:
         near_ties["oracle_sample"] = check_sampled_selection(w, cpu.pop("_sample"), idx_h[0, 0])
-    # the recorded ncu traffic belongs to the group-shared launch (two 128-row tiles per CTA)
-    traffic = None if args.per_qhead else profiled_traffic("attn_prefill_gqa128k.json", ATTN_SOURCES)
+    # the recorded ncu traffic belongs to the group-shared launch of the full-length 128K workload
+    headline = args.workload == WORKLOAD and not args.seq and not args.per_qhead
+    traffic = profiled_traffic("attn_prefill_gqa128k.json", ATTN_SOURCES) if headline else None
     config = config_dict(w, world)
     if args.per_qhead:
         config["workload"] += ", per-query-head selection"
@@ -413,7 +427,7 @@ def run_gpu(args, world, rank, local):
             "attention_tflops": achieved,
         },
         "roofline": {"bound": "tensor",
-                     "kernel": "attn_prefill_kernel<128,64,%d>" % (1 if args.per_qhead else 2), "achieved": achieved,
+                     "kernel": attention_kernel_name(shape), "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                      "peak_source": f"{how} bf16 dense (burst)", "traffic": traffic,
                      "flops_per_launch": attn_flops},

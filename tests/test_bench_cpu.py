@@ -53,3 +53,17 @@ def test_bench_selection_report_helpers():
                 idx[0, kvh, qi, 0] = j
     rec = bench.needle_recall(w, idx)
     assert rec["planted"] == 16 * w.heads_kv and rec["selected"] == 8 * w.heads_kv
+
+
+def test_bench_names_the_attention_kernel_the_library_launches():
+    """The roofline's kernel label follows the launcher's rule: two 128-row tiles per CTA for the
+    GQA groups of 64-token blocks, two units per CTA for units of at most 128 rows."""
+    import bench
+    import workloads
+    import block_sparse_long_pisa_b200 as pisa
+    name = lambda n, per=0: bench.attention_kernel_name(pisa.Shape.of(workloads.WORKLOADS[n], select_per_qhead=per))
+    assert name("gqa128k") == "attn_prefill_kernel<128,64,2>"
+    assert name("gqa128k", 1) == "attn_prefill_dual_kernel<128,64>"
+    assert name("causal32k") == "attn_prefill_dual_kernel<128,64>"
+    assert name("long1m") == "attn_prefill_dual_kernel<128,128>"
+    assert name("tiny") == "attn_prefill_dual_kernel<64,64>"
