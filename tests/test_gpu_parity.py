@@ -349,6 +349,28 @@ def test_capacity_pyramid_build_and_append(cuda_device):
                 gu.assert_pyramid_close(got[b, h], ref, offs)
 
 
+def test_pyramid_top_levels_past_the_shared_memory_limit(cuda_device):
+    """One plane of 21,000 key blocks: above the 64-block subtrees the pyramid has 441 rows
+    (225 KB at head dim 128), more than the top-level kernel keeps in shared memory, so it forms
+    those levels from global memory. The two-launch build equals the per-level path (an append
+    from an empty cache) bit for bit, and the oracle within the pyramid tolerance."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    n0, D = 21000, 128
+    shape = pisa.Shape(1, 1, 1, n0 * 64, n0 * 64, D, 64, 4, 64, causal=1)
+    sizes, offs = pisa.level_layout(shape)
+    assert sum(sizes[3:]) * D * 4 > 160 * 1024
+    gen = torch.Generator(device=cuda_device).manual_seed(1234)
+    k = torch.randn((1, 1, n0 * 64, D), generator=gen, device=cuda_device).to(torch.bfloat16)
+    built = pisa.build_pyramid(shape, k)
+    appended = torch.zeros_like(built)
+    pisa.append_pyramid(shape, k, appended, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(built, appended)
+    levels = oracle.build_pyramid(gu.host_f32(k)[0, 0], 64, 4)
+    gu.assert_pyramid_close(gu.host_f32(built)[0, 0], levels, offs)
+
+
 @pytest.mark.parametrize("forced", [0, 3])
 def test_decode_with_spare_capacity(forced, cuda_device):
     """Decode over a partly filled cache (spare rows hold NaN) matches the oracle's decode at the
