@@ -661,13 +661,10 @@ static bool launch_dq(const BwdParams& p, int32_t batch, cudaStream_t st) {
     if (!make_tmap_2d(&tq, p.Q, qrows, D, BLK) || !make_tmap_2d(&tdo, p.dO, qrows, D, BLK) ||
         !make_tmap_2d(&tk, p.K, krows, D, BLK) || !make_tmap_2d(&tv, p.V, krows, D, BLK))
         return false;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dq_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kRSmem)) != cudaSuccess)
-            return false;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!configure_smem_once(reinterpret_cast<const void*>(bwd_dq_tc_kernel<D, BLK>), static_cast<int>(kRSmem),
+                             configured))
+        return false;
     // 128 rows: two heads of 64-token blocks (one head, 64 rows, when the group is odd), or one head
     // of 128-token blocks
     const int gsel = p.per_qhead ? 1 : p.g;
@@ -694,13 +691,10 @@ static bool launch_dkdv(const BwdParams& p, int32_t batch, cudaStream_t st) {
     if (!make_tmap_2d(&tq, p.Q, qrows, D, kTB) || !make_tmap_2d(&tdo, p.dO, qrows, D, kTB) ||
         !make_tmap_2d(&tk, p.K, krows, D, kTB) || !make_tmap_2d(&tv, p.V, krows, D, kTB))
         return false;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kSmem)) != cudaSuccess)
-            return false;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!configure_smem_once(reinterpret_cast<const void*>(bwd_dkdv_tc_kernel<D, BLK>), static_cast<int>(kSmem),
+                             configured))
+        return false;
     // one CTA per 64 keys: a 128-key block is taken as its two halves
     bwd_dkdv_tc_kernel<D, BLK><<<dim3(p.n0 * (BLK / kTB), p.Hkv, batch), kThreads, kSmem, st>>>(tq, tdo, tk, tv, p);
     return cudaGetLastError() == cudaSuccess;

@@ -605,13 +605,9 @@ template <int D, int BLK, int NM>
 static bool launch_variant(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const AttnParams& p,
                            dim3 grid, cudaStream_t st) {
     using C = PrefillCfg<D, BLK, NM>;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(attn_prefill_kernel<D, BLK, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM) != cudaSuccess)
-            return false;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!configure_smem_once(reinterpret_cast<const void*>(attn_prefill_kernel<D, BLK, NM>), C::SMEM, configured))
+        return false;
     attn_prefill_kernel<D, BLK, NM><<<grid, C::THREADS, C::SMEM, st>>>(q, k, v, p);
     return cudaGetLastError() == cudaSuccess;
 }

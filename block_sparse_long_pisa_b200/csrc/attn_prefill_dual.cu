@@ -587,13 +587,9 @@ template <int D, int BLK>
 static bool launch_dual(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const AttnParams& p,
                         dim3 grid, cudaStream_t st) {
     using C = DualCfg<D, BLK>;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(attn_prefill_dual_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM) != cudaSuccess)
-            return false;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!configure_smem_once(reinterpret_cast<const void*>(attn_prefill_dual_kernel<D, BLK>), C::SMEM, configured))
+        return false;
     grid.x = (grid.x + 1) / 2;  // two query blocks per CTA
     attn_prefill_dual_kernel<D, BLK><<<grid, C::THREADS, C::SMEM, st>>>(q, k, v, p);
     return cudaGetLastError() == cudaSuccess;

@@ -11,6 +11,16 @@
 
 namespace pisa {
 
+bool configure_smem_once(const void* func, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return true;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
+
 static thread_local int32_t g_launches = 0;
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }

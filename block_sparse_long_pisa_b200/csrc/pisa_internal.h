@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include <cuda.h>
 
 #include "pisa.h"
@@ -232,6 +234,11 @@ bool launch_bwd_dkdv_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 bool bwd_dq_tc_supported(const BwdParams& p);
 bool launch_bwd_dq_tc(const BwdParams& p, int32_t batch, cudaStream_t st);
 // 2-D TMA view [rows, D] of a bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// device: the attribute belongs to each device's copy of the kernel, so a process that drives
+// several GPUs sets it on each. `done` holds one bit per device (devices 64 and up set it on
+// every call).
+bool configure_smem_once(const void* func, int bytes, std::atomic<uint64_t>& done);
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows);
 // 2-D TMA view [rows, D] of an fp32 tensor, boxes of 32 columns x 128 rows, 128-byte swizzle.
 bool make_tmap_2d_f32(CUtensorMap* m, const void* ptr, int64_t rows, int D);

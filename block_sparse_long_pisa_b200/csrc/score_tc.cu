@@ -214,14 +214,12 @@ bool launch_score_tc(const SelectParams& p, dim3 grid, cudaStream_t st) {
     CUtensorMap tq, tn;
     if (!make_tmap_2d_f32(&tq, p.qsplit, 2 * qrows, p.D) || !make_tmap_2d_f32(&tn, p.nsplit, 2 * nrows, p.D))
         return false;
-    static bool configured[2] = {false, false};
+    static std::atomic<uint64_t> configured[2] = {};
     const int k = p.D == 64 ? 0 : 1;
-    if (!configured[k]) {
-        if (cudaFuncSetAttribute(k == 0 ? score_tc_kernel<64> : score_tc_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem) != cudaSuccess)
-            return false;
-        configured[k] = true;
-    }
+    if (!configure_smem_once(k == 0 ? reinterpret_cast<const void*>(score_tc_kernel<64>)
+                                    : reinterpret_cast<const void*>(score_tc_kernel<128>),
+                             kStSmem, configured[k]))
+        return false;
     if (k == 0)
         score_tc_kernel<64><<<grid, kStThreads, kStSmem, st>>>(tq, tn, p);
     else
