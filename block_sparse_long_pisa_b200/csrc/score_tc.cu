@@ -2,7 +2,9 @@
 // pyramide", PISA page): every query-block summary of one selection row
 // against every eligible pyramid node of the levels the descent can visit, as
 // fp32 dot products q . node, written to the score plane that descent_kernel
-// reads (same tiling, same plane, same eligibility rule as the FFMA tiles).
+// reads. A tile is skipped when none of its nodes is eligible for any of its
+// query blocks at its level (a query block needs level l only when its descent
+// starts at l or above, and only nodes up to its last eligible one).
 //
 // One CTA per 128 query blocks x 128 nodes. Every fp32 operand value x enters
 // as a tf32 head h (x with its 13 low mantissa bits cleared) and the exact fp32
