@@ -1,0 +1,90 @@
+"""A seeded sweep over random supported shapes, GPU against the oracle through the C ABI.
+
+The named cases of the other GPU tests pick one shape per kernel variant; this sweep draws
+shapes at random inside the library's limits (head dim 64/128, key blocks 64/128, pooling
+factor 2/4/8, group size 1-8, 1-2 KV heads and sequences, 2-40 key blocks so that pyramids are
+ragged, K from 1 to beyond the eligible blocks, causal or not, prefill or decode, shared or
+per-query-head selection, forced sink and local blocks) so that a dispatch or index error tied
+to one combination shows. Each shape: pyramid planes, selection rows (equal to the oracle's or
+an admissible near-tie resolution), O and LSE on the GPU's own selection; every third prefill
+shape also runs the backward against the oracle's gradients.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+REL_MAX, REL_MEAN = 2e-2, 1e-3   # backward tolerance, as in test_gpu_backward.py
+
+
+def _draw(n=40, seed=2024):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for k in range(n):
+        D = int(rng.choice([64, 128]))
+        blk = int(rng.choice([64, 128]))
+        f = int(rng.choice([2, 4, 8]))
+        hkv = int(rng.integers(1, 3))
+        decode = bool(rng.random() < 0.25)
+        g = int(rng.choice([1, 2, 3, 4, 8]))
+        nb = int(rng.integers(2, 41))
+        causal = 0 if decode else int(rng.random() < 0.6)
+        topk = int(rng.integers(1, nb + 3))
+        batch = int(rng.integers(1, 3))
+        per_q = bool(rng.random() < 0.25)
+        forced = int(rng.choice([0, 0, 1, 2, 3]))
+        keys = str(rng.choice(["iid", "clustered"]))
+        w = workloads.Workload(f"rand{k}-d{D}-b{blk}-f{f}-g{g}-nb{nb}-k{topk}{'-dec' if decode else ''}"
+                               f"{'-causal' if causal else ''}{'-perq' if per_q else ''}-forced{forced}",
+                               batch, hkv * g, hkv, 1 if decode else nb * blk, nb * blk, D, blk, f, topk, causal,
+                               keys, 700 + k)
+        cases.append((w, per_q, forced))
+    return cases
+
+
+CASES = _draw()
+
+
+@pytest.mark.parametrize("case", range(len(CASES)), ids=[c[0].name for c in CASES])
+def test_random_shape_matches_oracle(case, cuda_device):
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w, per_q, forced = CASES[case]
+    shape = pisa.Shape.of(w, select_per_qhead=int(per_q), forced_blocks=forced)
+    q, k, v = (gu.to_device(w, t, cuda_device) for t in ("q", "k", "v"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, k, v, ws, idx=True)
+    pyr = pisa.build_pyramid(shape, k)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, w.name)
+    Q, K, V = (gu.host_f32(x) for x in (q, k, v))
+    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_q, forced=forced)
+    _, offs = pisa.level_layout(shape)
+    pyr_h = gu.host_f32(pyr)
+    for b in range(w.batch):
+        for h in range(w.heads_kv):
+            gu.assert_pyramid_close(pyr_h[b, h], ref["pyramid"][b][h], offs)
+    idx_h = idx.cpu().numpy()
+    gu.check_selection(idx_h, ref, w, per_qhead=per_q, forced=forced)
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_q,
+                           idx_override=idx_h)
+    gu.assert_output_close(gu.host_f32(o), ref_o["O"], gu.host_f32(lse), ref_o["lse"], w.name)
+    if w.decode or case % 3 != 0:
+        return
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1000)
+    do = torch.randn(tuple(q.shape), generator=g).to(torch.bfloat16).to(cuda_device)
+    ws_b = torch.zeros(pisa.backward_workspace_size(shape), dtype=torch.uint8, device=cuda_device)
+    dq, dk, dv = pisa.sparse_attention_backward(shape, q, k, v, o, lse, do, idx, ws=ws_b)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws_b, "backward")
+    grads = oracle.backward(Q, K, V, gu.host_f32(do), idx_h, w.block, bool(w.causal), per_qhead=per_q)
+    for name, got in (("dQ", dq), ("dK", dk), ("dV", dv)):
+        got = gu.host_f32(got).astype(np.float64)
+        want = grads[name]
+        scale = np.abs(want).max()
+        err = np.abs(got - want)
+        assert err.max() <= REL_MAX * scale, f"{w.name} {name}: max err {err.max():.3e} vs {scale:.3e}"
+        assert err.mean() <= REL_MEAN * scale, f"{w.name} {name}: mean err {err.mean():.3e} vs {scale:.3e}"
