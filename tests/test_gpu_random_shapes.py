@@ -7,7 +7,8 @@ ragged, K from 1 to beyond the eligible blocks, causal or not, prefill or decode
 per-query-head selection, forced sink and local blocks) so that a dispatch or index error tied
 to one combination shows. Each shape: pyramid planes, selection rows (equal to the oracle's or
 an admissible near-tie resolution), O and LSE on the GPU's own selection; every third prefill
-shape also runs the backward against the oracle's gradients.
+shape also runs the backward against the oracle's gradients. A second test runs the selection of
+every shape under random per-level budgets.
 """
 import numpy as np
 import pytest
@@ -88,3 +89,28 @@ def test_random_shape_matches_oracle(case, cuda_device):
         err = np.abs(got - want)
         assert err.max() <= REL_MAX * scale, f"{w.name} {name}: max err {err.max():.3e} vs {scale:.3e}"
         assert err.mean() <= REL_MEAN * scale, f"{w.name} {name}: mean err {err.mean():.3e} vs {scale:.3e}"
+
+
+@pytest.mark.parametrize("case", range(len(CASES)), ids=[c[0].name for c in CASES])
+def test_random_level_budgets_match_oracle(case, cuda_device):
+    """The same shapes with random per-level budgets K_l (level 0 keeps K; coarser levels keep
+    between 1 and twice K nodes, capped by the level's size): every selection row equals the
+    oracle's descent under those budgets, or is an admissible near-tie resolution of it."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w, per_q, forced = CASES[case]
+    shape = pisa.Shape.of(w, select_per_qhead=int(per_q), forced_blocks=forced)
+    sizes, _ = pisa.level_layout(shape)
+    rng = np.random.default_rng(9000 + case)
+    budgets = [w.topk] + [int(rng.integers(1, max(1, min(n, 2 * w.topk)) + 1)) for n in sizes[1:]]
+    q, k = (gu.to_device(w, t, cuda_device) for t in ("q", "k"))
+    ws = pisa.new_workspace(shape, cuda_device)
+    pyr = pisa.build_pyramid(shape, k)
+    idx = pisa.select_blocks(shape, q, pyr, ws, level_budget=budgets)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, w.name)
+    Q, K = gu.host_f32(q), gu.host_f32(k)
+    ref = oracle.forward(Q, K, K, w.block, w.factor, w.topk, bool(w.causal), per_qhead=per_q, budgets=budgets,
+                         forced=forced)
+    gu.check_selection(idx.cpu().numpy(), ref, w, per_qhead=per_q, budgets=budgets, forced=forced,
+                       what=f"{w.name} budgets {budgets}")
