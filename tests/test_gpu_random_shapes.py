@@ -8,7 +8,8 @@ per-query-head selection, forced sink and local blocks) so that a dispatch or in
 to one combination shows. Each shape: pyramid planes, selection rows (equal to the oracle's or
 an admissible near-tie resolution), O and LSE on the GPU's own selection; every third prefill
 shape also runs the backward against the oracle's gradients. A second test runs the selection of
-every shape under random per-level budgets.
+every shape under random per-level budgets; a third puts the decode shapes in a cache with spare
+capacity and checks the incremental pyramid against a fresh build.
 """
 import numpy as np
 import pytest
@@ -114,3 +115,49 @@ def test_random_level_budgets_match_oracle(case, cuda_device):
                          forced=forced)
     gu.check_selection(idx.cpu().numpy(), ref, w, per_qhead=per_q, budgets=budgets, forced=forced,
                        what=f"{w.name} budgets {budgets}")
+
+
+DECODE_CASES = [c for c, (w, _, _) in enumerate(CASES) if w.decode]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=[CASES[c][0].name for c in DECODE_CASES])
+def test_random_decode_with_spare_capacity_and_append(case, cuda_device):
+    """The sweep's decode shapes in a cache with spare capacity (1-20 blocks, rows past the
+    length hold NaN): decode matches the oracle at the cache's length, and a pyramid built at a
+    shorter length and appended up to it equals the one built at it, bit for bit."""
+    import torch
+    import block_sparse_long_pisa_b200 as pisa
+    w, per_q, forced = CASES[case]
+    rng = np.random.default_rng(9500 + case)
+    cap = w.seq_kv + int(rng.integers(1, 21)) * w.block
+    k, v = (gu.to_device(w, t, cuda_device) for t in ("k", "v"))
+    kc, vc = (torch.full((w.batch, w.heads_kv, cap, w.head_dim), float("nan"), dtype=torch.bfloat16,
+                         device=cuda_device) for _ in range(2))
+    kc[:, :, :w.seq_kv] = k
+    vc[:, :, :w.seq_kv] = v
+    q = gu.to_device(w, "q", cuda_device)
+    shape = pisa.Shape.of(w, select_per_qhead=int(per_q), forced_blocks=forced, kv_capacity=cap)
+    ws = pisa.new_workspace(shape, cuda_device)
+    o, lse, idx = pisa.forward(shape, q, kc, vc, ws, idx=True)
+    torch.cuda.synchronize()
+    pisa.raise_on_device_error(ws, w.name)
+    Q, K, V = gu.host_f32(q), gu.host_f32(kc), gu.host_f32(vc)
+    ref = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, per_qhead=per_q, kv_len=w.seq_kv,
+                         forced=forced)
+    idx = idx.cpu().numpy()
+    gu.check_selection(idx, ref, w, per_qhead=per_q, forced=forced, kv_len=w.seq_kv)
+    ref_o = oracle.forward(Q, K, V, w.block, w.factor, w.topk, False, per_qhead=per_q, kv_len=w.seq_kv,
+                           idx_override=idx)
+    o, lse = gu.host_f32(o), gu.host_f32(lse)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    gu.assert_output_close(o, ref_o["O"], lse, ref_o["lse"], w.name)
+    # append: from a shorter length (a multiple of the block) up to the cache's length
+    n_old = int(rng.integers(0, w.seq_kv // w.block)) * w.block
+    kz = torch.nan_to_num(kc, nan=0.0)
+    at = lambda n: pisa.Shape.of(w.replace(seq_kv=n), select_per_qhead=int(per_q), kv_capacity=cap)
+    pyr = pisa.build_pyramid(at(n_old), kz) if n_old > 0 else \
+        torch.zeros(pisa.pyramid_size(at(w.seq_kv)) // 4, dtype=torch.float32, device=cuda_device)
+    pisa.append_pyramid(at(w.seq_kv), kz, pyr, n_old)
+    fresh = pisa.build_pyramid(at(w.seq_kv), kz)
+    torch.cuda.synchronize()
+    assert torch.equal(pyr.view(-1), fresh.view(-1)), (w.name, n_old)
