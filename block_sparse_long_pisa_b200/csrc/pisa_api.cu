@@ -248,11 +248,16 @@ static pisa_status query_summary(const Plan& pl, const void* Q, float* qbar, cud
     return PISA_OK;
 }
 
-static pisa_status select(const Plan& pl, const float* qbar, const float* pyr, const int32_t* budget,
+// Decode passes the query tokens (Q) and no summaries: the descent kernel forms each row's
+// summary itself. Prefill passes the summaries of query_summary.
+static pisa_status select(const Plan& pl, const float* qbar, const void* Q, const float* pyr, const int32_t* budget,
                           int32_t* idx, float* margin, uint8_t* ws, cudaStream_t st) {
     uint32_t* status = reinterpret_cast<uint32_t*>(ws);
     SelectParams sp{};
     sp.qbar = qbar;
+    sp.qtok = pl.decode ? static_cast<const __nv_bfloat16*>(Q) : nullptr;
+    sp.Hq = pl.Hq;
+    sp.qheads = pl.gsel;
     sp.pyr = pyr;
     sp.idx = idx;
     sp.margin = margin;
@@ -542,8 +547,8 @@ pisa_status pisa_select_blocks(const pisa_shape* shape, const void* Q, const flo
     uint8_t* w = static_cast<uint8_t*>(ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
-    if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
-    return select(pl, qbar, pyramid, level_budget, idx, margin, w, st);
+    if (!pl.decode && (s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
+    return select(pl, qbar, Q, pyramid, level_budget, idx, margin, w, st);
 }
 
 pisa_status pisa_sparse_attention(const pisa_shape* shape, const void* Q, const void* K, const void* V,
@@ -578,8 +583,8 @@ pisa_status pisa_forward(const pisa_shape* shape, const void* Q, const void* K, 
     float* qbar = reinterpret_cast<float*>(w + pl.ws_qbar);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + pl.ws_idx);
     if ((s = build_pyramid(pl, K, pyr, st)) != PISA_OK) return s;
-    if ((s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
-    if ((s = select(pl, qbar, pyr, nullptr, idx, nullptr, w, st)) != PISA_OK) return s;
+    if (!pl.decode && (s = query_summary(pl, Q, qbar, st)) != PISA_OK) return s;
+    if ((s = select(pl, qbar, Q, pyr, nullptr, idx, nullptr, w, st)) != PISA_OK) return s;
     return attention(pl, Q, K, V, idx, O, lse, w, st);
 }
 

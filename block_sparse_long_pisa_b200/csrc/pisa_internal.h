@@ -136,7 +136,9 @@ struct SubtreeParams {
 };
 
 struct SelectParams {
-    const float* qbar;          // fp32 [B, Hsel, nqb, D]
+    const float* qbar;          // fp32 [B, Hsel, nqb, D] (prefill)
+    const __nv_bfloat16* qtok;  // decode: the query tokens [B, Hq, 1, D], summarised by the kernel
+    int32_t Hq, qheads;         // decode: query heads, and heads averaged per selection row
     const float* pyr;           // fp32 [B, Hkv, total_nodes, D]
     int32_t* idx;               // int32 [B, Hsel, nqb, topk]
     float* margin;              // optional fp32 [B, Hsel, nqb]

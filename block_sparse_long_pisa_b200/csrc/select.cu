@@ -87,8 +87,29 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
     // of the set-up and the first level's node loads)
     const int sub = tid & 7;
     float4 qv[D / 32];
+    if (p.qtok != nullptr) {
+        // decode: the summary is the mean of the row's heads' tokens, formed here in the fp32 order
+        // of block_mean_kernel (a running sum over the heads from zero, the +0 its lane reduction
+        // adds, one multiply by the reciprocal of the head count), so it is the same bit for bit
+        const float inv = 1.0f / static_cast<float>(p.qheads);
+        const __nv_bfloat16* q0 =
+            p.qtok + (static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(hs) * p.qheads) * D + 4 * sub;
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) qv[k] = *reinterpret_cast<const float4*>(p.qbar + row * D + 32 * k + 4 * sub);
+        for (int k = 0; k < D / 32; ++k) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            for (int h = 0; h < p.qheads; ++h) {
+                const uint2 w = *reinterpret_cast<const uint2*>(q0 + static_cast<int64_t>(h) * D + 32 * k);
+                a0 += __uint_as_float(w.x << 16);
+                a1 += __uint_as_float(w.x & 0xFFFF0000u);
+                a2 += __uint_as_float(w.y << 16);
+                a3 += __uint_as_float(w.y & 0xFFFF0000u);
+            }
+            qv[k] = make_float4((a0 + 0.0f) * inv, (a1 + 0.0f) * inv, (a2 + 0.0f) * inv, (a3 + 0.0f) * inv);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) qv[k] = *reinterpret_cast<const float4*>(p.qbar + row * D + 32 * k + 4 * sub);
+    }
     // partial (straddling) node summaries, bottom-up, where some level has a partial node
     bool any_part = false;
     for (int l = 1; l < p.L; ++l) {
