@@ -215,25 +215,36 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
                     th_hi = 0xFFFFFFFFu;  // nothing is kept (finite scores never reach this word)
                     th_lo = 0xFFFFFFFFu;
                 } else if (nvalid > k_l) {
-                    // score word of the K_l-th largest key: the largest h with at least K_l words >= h
+                    // score-word threshold of the K_l-th largest key by MSB-first bisection: the
+                    // largest h with at least K_l words >= h, or, as soon as a tested h keeps
+                    // exactly K_l words, that h (the cut then falls between two distinct scores)
                     th_hi = 0;
                     for (int bit = 31; bit >= 0; --bit) {
                         const uint32_t c = th_hi | (1u << bit);
                         int cnt = 0;
                         for (int t = s0; t < s1; ++t) cnt += static_cast<uint32_t>(keys[t] >> 32) >= c;
-                        if (static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, cnt)) >= k_l) th_hi = c;
+                        const int tot = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, cnt));
+                        if (tot >= k_l) {
+                            th_hi = c;
+                            if (tot == k_l) break;
+                        }
                     }
                     int gt = 0, eq = 0;
-                    uint32_t below = 0;  // largest score word under th_hi: the (K_l+1)-th score if no tie
+                    uint32_t below = 0;            // largest score word under th_hi: the (K_l+1)-th score if no tie
+                    uint32_t kept_min = 0xFFFFFFFFu;  // smallest score word at or above th_hi: the K_l-th score
                     for (int t = s0; t < s1; ++t) {
                         const uint32_t h = static_cast<uint32_t>(keys[t] >> 32);
                         gt += h > th_hi;
                         eq += h == th_hi;
-                        if (h < th_hi) below = max(below, h);
+                        if (h < th_hi)
+                            below = max(below, h);
+                        else
+                            kept_min = min(kept_min, h);
                     }
                     gt = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, gt));
                     eq = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, eq));
                     below = __reduce_max_sync(0xFFFFFFFFu, below);
+                    kept_min = __reduce_min_sync(0xFFFFFFFFu, kept_min);
                     const int need = k_l - gt;  // kept among the keys whose score word is th_hi
                     th_lo = 0;
                     if (eq > need) {
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams 
                         below = th_hi;  // the (K_l+1)-th score equals the K_l-th
                     }
                     if (lane == 0) {
-                        const float a = order_bits_inv(th_hi);
+                        const float a = order_bits_inv(kept_min);
                         const float c = order_bits_inv(below);
                         const float rel = (a - c) / fmaxf(fmaxf(fabsf(a), fabsf(c)), 1e-30f);
                         s_margin = fminf(s_margin, rel);
