@@ -1,8 +1,10 @@
 // Pyramid-guided top-K selection ("La selection top-K guidee par la pyramide",
 // PISA page). One CTA of 128 threads per (batch, selection row, query block).
 //
-// 1. Each lane holds its slice of the query summary (fp32, computed by the
-//    pooling kernel), loaded from global memory alongside the first nodes.
+// 1. Each lane holds its slice of the query summary, loaded from global memory
+//    alongside the first nodes: for prefill the fp32 summary the pooling kernel
+//    computed; for decode the kernel forms it from the row's query tokens (the
+//    same fp32 arithmetic, so no separate summary launch).
 // 2. Causal: the node that straddles the query block at each level is
 //    summarised by the mean of its eligible level-0 blocks, built bottom-up
 //    from the pyramid (full children left of the straddling child, plus the
@@ -22,7 +24,8 @@
 //    1.3x and 2x as long, since fewer of them are resident per SM.) Candidates are ranked by
 //    a 64-bit key (order-preserving score bits, then inverted node index): higher score first
 //    and, on equal scores, lower index. One warp finds the K_l-th largest key by bisection with
-//    warp-wide counts (the score word first, the index word only when scores tie at the cut;
+//    warp-wide counts, stopping as soon as a threshold keeps exactly K_l candidates (the score
+//    word first, the index word only when scores tie at the cut;
 //    a CTA barrier per step costs several hundred cycles here) and compacts the kept
 //    candidates in candidate order. Candidates are produced in
 //    ascending node order at every level (the first scored level's eligible nodes, then the
