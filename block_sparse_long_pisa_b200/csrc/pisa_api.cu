@@ -116,6 +116,7 @@ pisa_status make_plan(const pisa_shape* s, Plan* p) {
         const int64_t dense = static_cast<int64_t>(p->total_nodes) / (p->causal ? 2 : 1);
         const int64_t sparse = p->lsize[p->L - 1] + static_cast<int64_t>(p->L - 1) * p->topk * p->f;
         p->dense_select = !p->decode && p->nqb >= kDenseSelectMinQBlocks &&
+                          static_cast<int64_t>(p->B) * p->Hsel * p->nqb > kSparseSelectMaxRows &&
                           dense <= static_cast<int64_t>(kDenseSelectMaxWorkRatio) * sparse;
     }
     p->ws_scores = o;

@@ -39,6 +39,11 @@ constexpr int kDecMaxBps = 16;
 // eligible node densely (the tiles are shared by 128 query blocks); fewer
 // query blocks (and decode) score only the descent's candidates.
 constexpr int kDenseSelectMinQBlocks = 16;
+// Prefill selections of at most this many rows (batch x selection heads x query blocks: one wave
+// of the per-row descent, four 128-thread CTAs on each of 148 SMs) run the per-row descent: its
+// one launch beats the dense path's three there (measured: 128 rows 0.048 -> 0.038 ms, 512 rows
+// 0.065 -> 0.056 ms; at 600 rows the dense path takes 0.070 ms, the per-row descent a second wave).
+constexpr int64_t kSparseSelectMaxRows = 592;
 // The dense scoring is used while it scores at most this many times the
 // candidates the sparse descent scores (it is ~5x cheaper per candidate);
 // past that (very long contexts) the sparse descent's O(N log N) work wins.

@@ -122,8 +122,9 @@ PISA_API pisa_status pisa_pyramid_size(const pisa_shape *shape, size_t *bytes);
  * pisa_sparse_attention need for this shape (one size serves all three).
  * The first 256 bytes are the device status word; zero them once when the
  * workspace is allocated (pisa_check_status clears them after each read).
- * Prefill with 16 or more query blocks, while scoring every eligible node is
- * cheaper than the sparse descent (up to about 1M tokens at block 128), also
+ * Prefill with 16 or more query blocks and more than 592 selection rows
+ * (batch * Hsel * nQB), while scoring every eligible node is cheaper than the
+ * sparse descent (up to about 1M tokens at block 128), also
  * holds an fp32 score plane of B * Hsel * qc * total_nodes values (Hsel =
  * heads_kv, or heads_q with select_per_qhead): the selection scores and
  * descends qc query blocks at a time, qc a multiple of 128 chosen so the plane

@@ -27,14 +27,19 @@ SMALL = {
                                  "clustered", 16),
     "gqa4-d64-noncausal": W("gqa4-d64-noncausal", 2, 8, 2, 18 * 64, 18 * 64, 64, 64, 4, 5, 0, "iid", 17),
     "gqa4-needle": W("gqa4-needle", 1, 8, 2, 256 * 64, 256 * 64, 128, 64, 4, 16, 1, "needle", 18),
-    # fewer query blocks than the dense-scoring threshold: the sparse descent runs for prefill
+    # fewer query blocks than the dense-scoring threshold: the sparse descent runs for prefill (as it
+    # does for every prefill of at most 592 selection rows, the shapes above included)
     "gqa4-causal-short": W("gqa4-causal-short", 2, 8, 2, 13 * 64, 13 * 64, 128, 64, 4, 3, 1, "iid", 23),
+    # more than 592 selection rows: the dense scoring and the warp descent
+    "gqa2-dense-640": W("gqa2-dense-640", 2, 16, 8, 40 * 64, 40 * 64, 128, 64, 4, 6, 1, "iid", 24),
+    "mha-d64-b128-dense": W("mha-d64-b128-dense", 2, 8, 8, 40 * 128, 40 * 128, 64, 128, 8, 9, 1, "clustered", 25),
     "decode-gqa4": W("decode-gqa4", 3, 8, 2, 1, 45 * 64, 128, 64, 4, 9, 0, "clustered", 19),
     "decode-d64-b128": W("decode-d64-b128", 2, 4, 4, 1, 40 * 128, 64, 128, 8, 6, 0, "iid", 20),
 }
 PER_QHEAD = {
     "perq-gqa4-causal": W("perq-gqa4-causal", 1, 8, 2, 21 * 64, 21 * 64, 128, 64, 4, 5, 1, "iid", 21),
     "perq-decode": W("perq-decode", 2, 8, 2, 1, 30 * 64, 128, 64, 4, 7, 0, "iid", 22),
+    "perq-gqa4-dense": W("perq-gqa4-dense", 1, 16, 4, 40 * 64, 40 * 64, 128, 64, 4, 5, 1, "iid", 26),
 }
 
 
@@ -139,11 +144,13 @@ def test_exact_ties_go_to_lower_index(cuda_device):
     assert np.array_equal(idx, ref["idx"])
 
 
-def test_full_budgets_equal_exhaustive_topk(cuda_device):
-    """level_budget = n_l at every coarse level: the descent is exhaustive top-K."""
+@pytest.mark.parametrize("name", ["gqa4-causal-ragged", "gqa2-dense-640"])
+def test_full_budgets_equal_exhaustive_topk(name, cuda_device):
+    """level_budget = n_l at every coarse level: the descent is exhaustive top-K (per-row and
+    dense selection paths)."""
     import torch
     import block_sparse_long_pisa_b200 as pisa
-    w = SMALL["gqa4-causal-ragged"]
+    w = SMALL[name]
     shape = pisa.Shape.of(w)
     q, k = (gu.to_device(w, t, cuda_device) for t in ("q", "k"))
     sizes, _ = pisa.level_layout(shape)
@@ -268,7 +275,8 @@ def test_growing_logits_rescale_running_max(causal, cuda_device):
 
 FORCED_CASES = [("tiny", 3), ("gqa4-causal-ragged", 1), ("gqa4-causal-ragged", 2), ("gqa4-causal-ragged", 3),
                 ("gqa4-causal-short", 3), ("decode-gqa4", 3), ("decode-d64-b128", 2), ("perq-gqa4-causal", 3),
-                ("mha-d128-b128-f8-causal", 1)]
+                ("mha-d128-b128-f8-causal", 1), ("gqa2-dense-640", 3), ("perq-gqa4-dense", 3),
+                ("mha-d64-b128-dense", 2)]
 
 
 @pytest.mark.parametrize("name,forced", FORCED_CASES)
@@ -296,7 +304,7 @@ def test_forced_blocks_match_oracle(name, forced, cuda_device):
 def test_forced_blocks_fill_the_budget(topk, cuda_device):
     """K no larger than the forced blocks: K = 1 keeps the sink alone, K = 2 the sink and the
     query's own block, on both selection paths."""
-    for name in ("gqa4-causal-ragged", "gqa4-causal-short"):
+    for name in ("gqa4-causal-ragged", "gqa4-causal-short", "gqa2-dense-640"):
         w = SMALL[name]
         _, _, ref, _, _, idx, _ = _run(w, cuda_device, topk=topk, forced=3)
         assert np.array_equal(idx, ref["idx"]), name
